@@ -1,0 +1,119 @@
+"""Seeded synthetic inputs for the GQA attention forward.
+
+This module holds no attention arithmetic: it only draws the tensors that both
+the CUDA path and the fp64 oracle are fed, so that the two sides see the same
+bits.  Everything is drawn on the CPU from ``torch.Generator`` seeded per
+workload, so a given (workload, seed) gives identical tensors on every machine
+with the same torch build.
+
+Recipe (per workload below):
+  * Q, K, V: ``randn`` in float32 times ``sigma``, rounded to bf16
+    (round-to-nearest-even, torch's cast);
+  * kv_len: all equal to the workload's length, or, for the batched decode,
+    ``randint`` uniform in [1, Tkv];
+  * K and V rows at positions >= kv_len (the padded capacity) are overwritten
+    with NaN where the workload asks for NaN padding, so that any read of a
+    padded row shows up in the output;
+  * sink: ``randn`` float32 per query head (already in the scaled-logit domain).
+
+The five named workloads are the shapes the pages measure or describe: the
+tiny prefill, the batched decode with ragged lengths, the short-query/long-KV
+prefill (AstrAI commit log, head-packing commit: G=8, B=16, q=16, kv=16k), the
+full causal prefill, and the wide-head decode with a sink and a length that is
+not a multiple of 128 (nvfp4-megamoe-kernel dsv4/kernels/attention commit log:
+head dims up to 512, sink logit, logical vs padded length).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, replace
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Tq: int
+    Tkv: int            # buffer capacity of K/V
+    d: int
+    sigma: float = 1.0  # std of Q, K, V
+    causal: bool = False
+    sink: bool = False
+    kv_len: int | None = None   # fixed logical length (None: = Tkv)
+    ragged: bool = False        # kv_len ~ U[1, Tkv] per batch
+    nan_pad: bool = False       # K/V rows >= kv_len are NaN
+    seed: int = 0
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+
+WORKLOADS = {
+    "tiny_prefill": Workload("tiny_prefill", B=1, Hq=4, Hkv=1, Tq=16, Tkv=128, d=64,
+                             seed=1001),
+    "batched_decode": Workload("batched_decode", B=16, Hq=32, Hkv=4, Tq=1, Tkv=16384, d=128,
+                               ragged=True, nan_pad=True, seed=1002),
+    "short_q_long_kv": Workload("short_q_long_kv", B=16, Hq=32, Hkv=4, Tq=16, Tkv=16384, d=128,
+                                causal=True, seed=1003),
+    "full_causal_prefill": Workload("full_causal_prefill", B=4, Hq=32, Hkv=8, Tq=4096, Tkv=4096,
+                                    d=128, causal=True, seed=1004),
+    "wide_head_sink_decode": Workload("wide_head_sink_decode", B=8, Hq=32, Hkv=1, Tq=4, Tkv=8192,
+                                      d=512, sigma=0.5, causal=True, sink=True, kv_len=8131,
+                                      nan_pad=True, seed=1005),
+}
+
+
+def shrink(w: Workload, **kw) -> Workload:
+    """A copy of a workload with some fields replaced (smaller parity cases)."""
+    return replace(w, **kw)
+
+
+@dataclass
+class Inputs:
+    q: torch.Tensor            # bf16 [B, Hq, Tq, d]
+    k: torch.Tensor            # bf16 [B, Hkv, Tkv, d]
+    v: torch.Tensor            # bf16 [B, Hkv, Tkv, d]
+    kv_lens: torch.Tensor | None   # int32 [B]
+    sink: torch.Tensor | None      # float32 [Hq]
+    scale: float
+    causal: bool
+
+
+def make_inputs(w: Workload, seed: int | None = None) -> Inputs:
+    """Draw the workload's tensors on the CPU."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed if seed is None else seed)
+
+    def normal(shape):
+        x = torch.randn(shape, generator=g, dtype=torch.float32)
+        if w.sigma != 1.0:
+            x.mul_(w.sigma)
+        return x.to(torch.bfloat16)
+
+    q = normal((w.B, w.Hq, w.Tq, w.d))
+    k = normal((w.B, w.Hkv, w.Tkv, w.d))
+    v = normal((w.B, w.Hkv, w.Tkv, w.d))
+    if w.ragged:
+        kv_lens = torch.randint(1, w.Tkv + 1, (w.B,), generator=g, dtype=torch.int32)
+    elif w.kv_len is not None:
+        kv_lens = torch.full((w.B,), w.kv_len, dtype=torch.int32)
+    else:
+        kv_lens = None
+    if w.nan_pad and kv_lens is not None:
+        for b in range(w.B):
+            n = int(kv_lens[b])
+            if n < w.Tkv:
+                k[b, :, n:, :] = float("nan")
+                v[b, :, n:, :] = float("nan")
+    sink = torch.randn((w.Hq,), generator=g, dtype=torch.float32) if w.sink else None
+    return Inputs(q=q, k=k, v=v, kv_lens=kv_lens, sink=sink, scale=w.scale, causal=w.causal)
+
