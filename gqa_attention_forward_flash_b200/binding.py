@@ -1,0 +1,144 @@
+"""Thin Python binding of the C ABI (include/gqa_attn.h), same names.
+
+Argument marshalling only: shapes come from the tensors, pointers from
+``data_ptr()``, the stream from torch's current CUDA stream.  Every step of the
+computation runs in the library's CUDA kernels; there is no fallback.  If the
+library is missing or cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgqa_attn.so")
+
+STATUS = {
+    0: "GQA_OK", -1: "GQA_ERR_NULL", -2: "GQA_ERR_SHAPE", -3: "GQA_ERR_ALIGN", -4: "GQA_ERR_SPLITS",
+    -5: "GQA_ERR_CUDA", -6: "GQA_ERR_TIMEOUT", -7: "GQA_ERR_UNSUPPORTED", -8: "GQA_ERR_KVLEN",
+}
+MAX_SPLITS = 256
+
+# exported names and their C signatures (restype, argtypes)
+_P, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+SIGNATURES = {
+    "gqa_attention_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "gqa_attention_fwd_partial": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P, _P]),
+    "gqa_splitkv_combine": (_I, [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "gqa_get_device_error": (_I, [_P]),
+    "gqa_status_string": (ctypes.c_char_p, [_I]),
+    "gqa_version": (_I, []),
+}
+
+_lib = None
+
+
+class GQAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__("%s failed: %s (%d)" % (fn, STATUS.get(status, "?"), status))
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError("libgqa_attn.so is not built; run `python -m gqa_attention_forward_flash_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise GQAError(fn, rc)
+
+
+def _need(t, dtype, name, ndim):
+    if t.dtype != dtype or t.dim() != ndim or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError("%s must be a contiguous CUDA %s tensor with %d dims" % (name, dtype, ndim))
+
+
+def gqa_attention_fwd(q, k, v, kv_lens=None, sink=None, out=None, lse=None, scale=None, causal=False,
+                      stream=None):
+    """O (and lse) of the GQA forward.  q [B,Hq,Tq,d], k/v [B,Hkv,Tkv,d] bf16;
+    kv_lens int32 [B] or None; sink fp32 [Hq] or None.  Returns (out, lse)."""
+    _need(q, torch.bfloat16, "q", 4)
+    _need(k, torch.bfloat16, "k", 4)
+    _need(v, torch.bfloat16, "v", 4)
+    B, Hq, Tq, d = q.shape
+    _, Hkv, Tkv, _ = k.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=q.device)
+    if kv_lens is not None:
+        _need(kv_lens, torch.int32, "kv_lens", 1)
+    if sink is not None:
+        _need(sink, torch.float32, "sink", 1)
+    if scale is None:
+        scale = d ** -0.5
+    rc = load().gqa_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_lens), _ptr(sink), _ptr(out), _ptr(lse),
+                                  B, Hq, Hkv, Tq, Tkv, d, float(scale), int(bool(causal)), _stream(stream))
+    _check("gqa_attention_fwd", rc)
+    return out, lse
+
+
+def gqa_attention_fwd_partial(q, k, v, kv_lens=None, scale=None, causal=False, num_splits=2, o_part=None,
+                              lse_part=None, stream=None):
+    """Split partials (no combine, no sink): o_part fp32 [B,Hq,Tq,S,d], lse_part fp32 [B,Hq,Tq,S]."""
+    B, Hq, Tq, d = q.shape
+    _, Hkv, Tkv, _ = k.shape
+    if o_part is None:
+        o_part = torch.empty((B, Hq, Tq, num_splits, d), dtype=torch.float32, device=q.device)
+    if lse_part is None:
+        lse_part = torch.empty((B, Hq, Tq, num_splits), dtype=torch.float32, device=q.device)
+    if scale is None:
+        scale = d ** -0.5
+    rc = load().gqa_attention_fwd_partial(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_lens), B, Hq, Hkv, Tq, Tkv, d,
+                                          float(scale), int(bool(causal)), int(num_splits), _ptr(o_part),
+                                          _ptr(lse_part), _stream(stream))
+    _check("gqa_attention_fwd_partial", rc)
+    return o_part, lse_part
+
+
+def gqa_splitkv_combine(o_part, lse_part, sink=None, out=None, lse=None, stream=None):
+    """LSE combine of [B,Hq,Tq,S,d] partials into bf16 out [B,Hq,Tq,d] and lse."""
+    B, Hq, Tq, S, d = o_part.shape
+    if out is None:
+        out = torch.empty((B, Hq, Tq, d), dtype=torch.bfloat16, device=o_part.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=o_part.device)
+    rc = load().gqa_splitkv_combine(_ptr(o_part), _ptr(lse_part), S, _ptr(sink), _ptr(out), _ptr(lse),
+                                    B, Hq, Tq, d, _stream(stream))
+    _check("gqa_splitkv_combine", rc)
+    return out, lse
+
+
+def gqa_get_device_error(stream=None) -> int:
+    return load().gqa_get_device_error(_stream(stream))
+
+
+def gqa_status_string(status: int) -> str:
+    return load().gqa_status_string(int(status)).decode()
+
+
+def gqa_version() -> int:
+    return load().gqa_version()

@@ -1,0 +1,331 @@
+// gqa_attn.cu -- host side of the C ABI declared in include/gqa_attn.h:
+// argument validation, kernel choice per head dim, TMA descriptors, the
+// per-device scratch for split partials, launches.
+//
+// Validation follows the rules the AstrAI commit log lists for its attention
+// bindings (q-head / kv-head divisibility, head-dim contiguity, split-KV scratch
+// layout) and its rule not to swallow cudaFuncSetAttribute failures.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "gqa_attn.h"
+#include "gqa_fwd_kernel.cuh"
+
+namespace gqa {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxCtas = 512;  // the stream-K combine keeps its slot list in 512 entries
+
+struct DeviceState {
+    bool init = false;
+    int sm_count = 0;
+    int cc_major = 0, cc_minor = 0;
+    long long clock_khz = 0;
+    int* err = nullptr;          // device error word
+    void* scratch = nullptr;     // stream-K slots + meta
+    size_t scratch_bytes = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_state(DeviceState** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GQA_ERR_CUDA;
+    DeviceState& s = g_dev[dev];
+    if (!s.init) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return GQA_ERR_CUDA;
+        s.sm_count = prop.multiProcessorCount;
+        s.cc_major = prop.major;
+        s.cc_minor = prop.minor;
+        int khz = 0;
+        if (cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev) != cudaSuccess || khz <= 0) khz = 2000000;
+        s.clock_khz = khz;
+        if (cudaMalloc(&s.err, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
+        if (cudaMemset(s.err, 0, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
+        s.init = true;
+    }
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return GQA_ERR_CUDA;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    *out = &s;
+    return GQA_OK;
+}
+
+// 2-D bf16 view [rows, cols] with a (64 x box_rows) box and the 128-byte swizzle.
+int make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int Tq, int Tkv, int d) {
+    if (B < 0 || Tq < 0 || Hq <= 0 || Hkv <= 0 || Tkv < 1) return GQA_ERR_SHAPE;
+    if (Hq % Hkv != 0) return GQA_ERR_SHAPE;
+    if (d != 64 && d != 128 && d != 256 && d != 512) return GQA_ERR_UNSUPPORTED;
+    const long long qrows = static_cast<long long>(B) * Hq * Tq;
+    const long long kvrows = static_cast<long long>(B) * Hkv * Tkv;
+    if (qrows + BM >= (1ll << 31) || kvrows + 256 >= (1ll << 31)) return GQA_ERR_SHAPE;
+    if (B == 0 || Tq == 0) return GQA_OK;
+    if (!q || !k || !v) return GQA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return GQA_ERR_ALIGN;
+    return GQA_OK;
+}
+
+void fill_params(Params& p, int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale, int causal,
+                 const int32_t* kv_lens, const float* sink, void* out, float* lse, int BN, long long timeout) {
+    std::memset(&p, 0, sizeof p);
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Tq = Tq;
+    p.Tkv = Tkv;
+    p.d = d;
+    p.G = Hq / Hkv;
+    p.R = p.G * Tq;
+    p.QT = (p.R + BM - 1) / BM;
+    p.U = B * Hkv;
+    p.W = static_cast<long long>(p.U) * p.QT;
+    p.causal = causal ? 1 : 0;
+    p.BN = BN;
+    p.scale_log2 = scale * LOG2E;
+    p.kv_lens = kv_lens;
+    p.sink = sink;
+    p.out = reinterpret_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.timeout_cycles = timeout;
+}
+
+// Kernel configurations per head dim (shared memory budget in FwdCfg).
+using Cfg64 = FwdCfg<64, 128, 4, 2>;
+using Cfg128 = FwdCfg<128, 128, 2, 2>;
+using Cfg256 = FwdCfg<256, 64, 2, 1>;
+
+template <class C>
+int launch_fwd(const Params& p0, const void* q, const void* k, const void* v, int grid, cudaStream_t stream) {
+    static bool attr_done[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_done[dev]) {
+        if (cudaFuncSetAttribute(gqa_fwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+            cudaSuccess)
+            return GQA_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    CUtensorMap tq, tk, tv;
+    Params p = p0;
+    // a box never taller than the tensor; rows a short box leaves unwritten are
+    // padding rows (query rows past the group, or key rows past kv_len, which the
+    // kernel zeroes in V and masks in S)
+    const uint64_t qrows = static_cast<uint64_t>(p.B) * p.Hq * p.Tq;
+    const uint64_t kvrows = static_cast<uint64_t>(p.B) * p.Hkv * p.Tkv;
+    p.q_box_rows = qrows < static_cast<uint64_t>(BM) ? static_cast<int>(qrows) : BM;
+    p.kv_box_rows = kvrows < static_cast<uint64_t>(C::BN) ? static_cast<int>(kvrows) : C::BN;
+    int rc = make_tmap(&tq, q, qrows, C::D, p.q_box_rows);
+    if (rc) return rc;
+    rc = make_tmap(&tk, k, kvrows, C::D, p.kv_box_rows);
+    if (rc) return rc;
+    rc = make_tmap(&tv, v, kvrows, C::D, p.kv_box_rows);
+    if (rc) return rc;
+    gqa_fwd_kernel<C><<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+int bn_for(int d) {
+    switch (d) {
+        case 64: return Cfg64::BN;
+        case 128: return Cfg128::BN;
+        case 256: return Cfg256::BN;
+        default: return 0;
+    }
+}
+
+int dispatch_fwd(const Params& p, const void* q, const void* k, const void* v, int grid, cudaStream_t stream) {
+    switch (p.d) {
+        case 64: return launch_fwd<Cfg64>(p, q, k, v, grid, stream);
+        case 128: return launch_fwd<Cfg128>(p, q, k, v, grid, stream);
+        case 256: return launch_fwd<Cfg256>(p, q, k, v, grid, stream);
+        default: return GQA_ERR_UNSUPPORTED;
+    }
+}
+
+int dispatch_combine_streamk(const Params& p, int grid, cudaStream_t stream) {
+    switch (p.d) {
+        case 64: gqa_combine_streamk_kernel<64><<<grid, 256, 0, stream>>>(p); break;
+        case 128: gqa_combine_streamk_kernel<128><<<grid, 256, 0, stream>>>(p); break;
+        case 256: gqa_combine_streamk_kernel<256><<<grid, 256, 0, stream>>>(p); break;
+        default: return GQA_ERR_UNSUPPORTED;
+    }
+    return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+long long timeout_cycles(const DeviceState& s) {
+    // about one second of SM clock, overridable for tests (GQA_WAIT_TIMEOUT_MS)
+    long long ms = 1000;
+    if (const char* e = std::getenv("GQA_WAIT_TIMEOUT_MS")) {
+        long long v = std::atoll(e);
+        if (v > 0) ms = v;
+    }
+    return s.clock_khz * ms;
+}
+
+int ensure_scratch(DeviceState& s, size_t bytes) {
+    if (s.scratch_bytes >= bytes) return GQA_OK;
+    if (s.scratch) {
+        // the old buffer may still be read by work queued on any stream
+        if (cudaDeviceSynchronize() != cudaSuccess) return GQA_ERR_CUDA;
+        cudaFree(s.scratch);
+        s.scratch = nullptr;
+        s.scratch_bytes = 0;
+    }
+    if (cudaMalloc(&s.scratch, bytes) != cudaSuccess) return GQA_ERR_CUDA;
+    s.scratch_bytes = bytes;
+    return GQA_OK;
+}
+
+}  // namespace
+}  // namespace gqa
+
+using namespace gqa;
+
+extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, const int32_t* kv_lens,
+                                 const float* sink, void* out, float* lse, int B, int Hq, int Hkv, int Tq,
+                                 int Tkv, int d, float scale, int causal, gqa_stream_t stream) {
+    int rc = check_common(q, k, v, B, Hq, Hkv, Tq, Tkv, d);
+    if (rc) return rc;
+    if (B == 0 || Tq == 0) return GQA_OK;
+    if (!out) return GQA_ERR_NULL;
+    if (!aligned16(out) || (lse && !aligned16(lse))) return GQA_ERR_ALIGN;
+    if (d == 512) return GQA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState* s = nullptr;
+    rc = get_state(&s);
+    if (rc) return rc;
+    if (s->cc_major != 10) return GQA_ERR_UNSUPPORTED;
+    Params p;
+    fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale, causal, kv_lens, sink, out, lse, bn_for(d), timeout_cycles(*s));
+    // grid: one CTA per SM; with host-known lengths never more CTAs than tiles
+    int NC = s->sm_count < kMaxCtas ? s->sm_count : kMaxCtas;
+    if (!kv_lens) {
+        long long tot = 0;
+        for (int qt = 0; qt < p.QT; ++qt) tot += qtile_ntiles(p, qt, Tkv);
+        tot *= p.U;
+        if (tot < NC) NC = static_cast<int>(tot);
+    }
+    if (NC < 1) NC = 1;
+    const size_t slot_o = static_cast<size_t>(2 * NC) * BM * d * sizeof(float);
+    const size_t slot_l = static_cast<size_t>(2 * NC) * BM * sizeof(float);
+    const size_t meta = static_cast<size_t>(NC) * 4 * sizeof(long long);
+    rc = ensure_scratch(*s, slot_o + slot_l + meta);
+    if (rc) return rc;
+    char* base = static_cast<char*>(s->scratch);
+    p.mode = 0;
+    p.part_o = reinterpret_cast<float*>(base);
+    p.part_lse = reinterpret_cast<float*>(base + slot_o);
+    p.meta = reinterpret_cast<long long*>(base + slot_o + slot_l);
+    p.err = s->err;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    rc = dispatch_fwd(p, q, k, v, NC, st);
+    if (rc) return rc;
+    return dispatch_combine_streamk(p, NC, st);
+}
+
+extern "C" int gqa_attention_fwd_partial(const void* q, const void* k, const void* v, const int32_t* kv_lens,
+                                         int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale, int causal,
+                                         int num_splits, float* o_part, float* lse_part, gqa_stream_t stream) {
+    int rc = check_common(q, k, v, B, Hq, Hkv, Tq, Tkv, d);
+    if (rc) return rc;
+    if (num_splits < 1 || num_splits > GQA_MAX_SPLITS) return GQA_ERR_SPLITS;
+    if (B == 0 || Tq == 0) return GQA_OK;
+    if (!o_part || !lse_part) return GQA_ERR_NULL;
+    if (!aligned16(o_part) || !aligned16(lse_part)) return GQA_ERR_ALIGN;
+    if (d == 512) return GQA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState* s = nullptr;
+    rc = get_state(&s);
+    if (rc) return rc;
+    if (s->cc_major != 10) return GQA_ERR_UNSUPPORTED;
+    Params p;
+    fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale, causal, kv_lens, nullptr, nullptr, nullptr, bn_for(d),
+                timeout_cycles(*s));
+    const long long grid = p.W * num_splits;
+    if (grid >= (1ll << 31)) return GQA_ERR_SHAPE;
+    p.mode = 1;
+    p.num_splits = num_splits;
+    p.part_o = o_part;
+    p.part_lse = lse_part;
+    p.err = s->err;
+    return dispatch_fwd(p, q, k, v, static_cast<int>(grid), reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int gqa_splitkv_combine(const float* o_part, const float* lse_part, int num_splits, const float* sink,
+                                   void* out, float* lse, int B, int Hq, int Tq, int d, gqa_stream_t stream) {
+    if (B < 0 || Hq <= 0 || Tq < 0 || d <= 0 || d % 4 != 0) return GQA_ERR_SHAPE;
+    if (num_splits < 1 || num_splits > GQA_MAX_SPLITS) return GQA_ERR_SPLITS;
+    if (B == 0 || Tq == 0) return GQA_OK;
+    if (!o_part || !lse_part || !out) return GQA_ERR_NULL;
+    if (!aligned16(o_part) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lse_part) & 3u)) return GQA_ERR_ALIGN;
+    const long long rows = static_cast<long long>(B) * Hq * Tq;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState* s = nullptr;
+    int rc = get_state(&s);
+    if (rc) return rc;
+    long long blocks = (rows + 7) / 8;
+    const long long cap = static_cast<long long>(s->sm_count) * 16;
+    if (blocks > cap) blocks = cap;
+    const size_t smem = static_cast<size_t>(8) * num_splits * sizeof(float);
+    gqa_combine_uniform_kernel<<<static_cast<int>(blocks), 256, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
+        o_part, lse_part, num_splits, sink, reinterpret_cast<__nv_bfloat16*>(out), lse, rows, Hq, Tq, d);
+    return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+extern "C" int gqa_get_device_error(gqa_stream_t stream) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState* s = nullptr;
+    int rc = get_state(&s);
+    if (rc) return rc;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return GQA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, s->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GQA_ERR_CUDA;
+    if (v != 0 && cudaMemset(s->err, 0, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
+    return v;
+}
+
+extern "C" const char* gqa_status_string(int status) {
+    switch (status) {
+        case GQA_OK: return "ok";
+        case GQA_ERR_NULL: return "a required pointer is NULL";
+        case GQA_ERR_SHAPE: return "invalid shape";
+        case GQA_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+        case GQA_ERR_SPLITS: return "num_splits out of range";
+        case GQA_ERR_CUDA: return "a CUDA call failed";
+        case GQA_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+        case GQA_ERR_UNSUPPORTED: return "unsupported head dim or GPU";
+        case GQA_ERR_KVLEN: return "a kv_lens value was outside [0, Tkv] and was clamped";
+        default: return "unknown status";
+    }
+}
+
+extern "C" int gqa_version(void) { return 100; }

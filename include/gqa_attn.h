@@ -1,0 +1,137 @@
+/*
+ * gqa_attn.h -- C ABI of the B200 (sm_100a) grouped-query-attention forward.
+ *
+ * The operation (one definition for every entry point below):
+ *
+ *   O = softmax( scale * Q K^T  + mask  [+ per-head sink logit] ) V
+ *
+ *   for batch b, query head h, query row i, with G = Hq / Hkv query heads
+ *   sharing each KV head and g = floor(h / G) the KV head that h reads
+ *   (contiguous grouping; AstrAI commit log, head-packing commit "pack
+ *   HB = min(G, WARPS) q heads per block"):
+ *     n   = kv_lens[b]  (logical length; rows n..Tkv-1 of the K/V buffers are
+ *           padding and never read into the result -- nvfp4-megamoe-kernel
+ *           dsv4/kernels/attention commit log, "logical vs padded N" commit)
+ *     visible keys j: 0 <= j < n and, when causal, j <= n - Tq + i
+ *           (causal mask aligned bottom-right against the logical length)
+ *     sink[h] is one extra logit with a zero value row, in the already-scaled
+ *           domain: it is never multiplied by `scale` (dsv4 attention commit
+ *           log, sink commit)
+ *     lse[b,h,i] = ln( sum_visible exp(s_j) + exp(sink[h]) ), natural log
+ *   A row with no visible key and no sink gets O = 0 and lse = -inf.  The
+ *   computation is tile by tile with an online-softmax (m, l, O) carry (dsv4
+ *   attention commit log, multi-tile commit: running max/sum rescale, O / l
+ *   once at the end); long key ranges are split over SMs and the partial
+ *   (O, lse) merged by an LSE combine (AstrAI commit log, split-KV scratch
+ *   validation commit; kernbench2 benches commit log, (m, l, O) merge commits).
+ *
+ * Layouts (all tensors contiguous, row-major, device memory unless stated):
+ *   q, out   bf16  [B, Hq,  Tq,  d]
+ *   k, v     bf16  [B, Hkv, Tkv, d]      Tkv = buffer capacity
+ *   kv_lens  int32 [B]                   or NULL (every n = Tkv)
+ *   sink     fp32  [Hq]                  or NULL (no sink)
+ *   lse      fp32  [B, Hq, Tq]           or NULL (not written)
+ *   o_part   fp32  [B, Hq, Tq, S, d]     (split partials, each normalised over its keys)
+ *   lse_part fp32  [B, Hq, Tq, S]        (natural log; -inf for a split with no key)
+ *
+ * Supported: d in {64, 128, 256, 512}; Hq % Hkv == 0; 1 <= Tkv; B*Hkv*Tkv and
+ * B*Hq*Tq below 2^31; every pointer 16-byte aligned.  B == 0 or Tq == 0 is a
+ * valid empty call.  kv_lens values outside [0, Tkv] are clamped to that range
+ * on the device and reported by gqa_get_device_error (GQA_ERR_KVLEN).
+ *
+ * Ownership and ordering: the caller owns every tensor.  Calls are
+ * asynchronous on `stream` (a cudaStream_t; NULL = the legacy default stream)
+ * and never synchronise the host.  gqa_attention_fwd keeps one scratch buffer
+ * per device for its split partials (grown on the host when a larger problem
+ * arrives, never freed before exit); calls on different streams of one device
+ * must therefore be ordered by the caller.
+ *
+ * Errors: every entry point returns a gqa_status.  Argument errors are found on
+ * the host before anything is launched.  Launch and attribute failures return
+ * GQA_ERR_CUDA (they are never swallowed -- AstrAI commit log, dynamic shared
+ * memory commit).  Waits inside the kernels are bounded: a wait that runs out
+ * records GQA_ERR_TIMEOUT in a device word, the kernel returns, and
+ * gqa_get_device_error reports it.
+ */
+#ifndef GQA_ATTN_H
+#define GQA_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *gqa_stream_t; /* the same handle type as cudaStream_t */
+
+typedef enum {
+    GQA_OK = 0,
+    GQA_ERR_NULL = -1,        /* a required pointer is NULL */
+    GQA_ERR_SHAPE = -2,       /* negative size, Hq % Hkv != 0, Tkv < 1, index overflow */
+    GQA_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned */
+    GQA_ERR_SPLITS = -4,      /* num_splits outside [1, GQA_MAX_SPLITS] */
+    GQA_ERR_CUDA = -5,        /* a CUDA runtime/driver call failed */
+    GQA_ERR_TIMEOUT = -6,     /* a bounded wait inside a kernel ran out (device-reported) */
+    GQA_ERR_UNSUPPORTED = -7, /* head dim not in {64,128,256,512}, or the GPU is not sm_100 */
+    GQA_ERR_KVLEN = -8        /* a kv_lens value was outside [0, Tkv] (device-reported, clamped) */
+} gqa_status;
+
+#define GQA_MAX_SPLITS 256
+
+/*
+ * The forward.  out and lse receive the attention defined above.  scale is the
+ * logit multiplier (1/sqrt(d) in the usual case); causal != 0 enables the
+ * bottom-right causal mask.
+ */
+int gqa_attention_fwd(const void *q, const void *k, const void *v, const int32_t *kv_lens,
+                      const float *sink, void *out, float *lse, int B, int Hq, int Hkv, int Tq,
+                      int Tkv, int d, float scale, int causal, gqa_stream_t stream);
+
+/*
+ * The split-KV half of the forward, with the split count forced by the caller
+ * (no combine, no sink).  For every query row the visible keys of its packed
+ * head group are cut into num_splits contiguous ranges; split s writes the
+ * attention over its range alone, normalised over that range, to
+ * o_part[b,h,i,s,:] and its log-sum-exp to lse_part[b,h,i,s] (-inf, with
+ * O = 0, for a range that holds no visible key).  gqa_splitkv_combine of these
+ * partials (with the sink) equals gqa_attention_fwd.  Only that combination is
+ * specified: where the cuts fall is an implementation choice.
+ */
+int gqa_attention_fwd_partial(const void *q, const void *k, const void *v, const int32_t *kv_lens,
+                              int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale,
+                              int causal, int num_splits, float *o_part, float *lse_part,
+                              gqa_stream_t stream);
+
+/*
+ * LSE combine of S = num_splits partials per row (the merge of softmax states
+ * over disjoint key sets; kernbench2 benches commit log, (m, l, O) merge and
+ * its associativity):
+ *   lse = ln( sum_s exp(lse_part[s]) + exp(sink[h]) ),
+ *   out = sum_s exp(lse_part[s] - lse) * o_part[s]       (bf16, round to nearest)
+ * sink may be NULL; lse may be NULL.  A row whose partials are all -inf and
+ * that has no sink gets out = 0, lse = -inf.
+ */
+int gqa_splitkv_combine(const float *o_part, const float *lse_part, int num_splits,
+                        const float *sink, void *out, float *lse, int B, int Hq, int Tq, int d,
+                        gqa_stream_t stream);
+
+/*
+ * Waits for `stream`, then returns (and clears) the first error a kernel of
+ * this library recorded on the current device since the last call: GQA_OK,
+ * GQA_ERR_TIMEOUT or GQA_ERR_KVLEN; GQA_ERR_CUDA if the synchronisation itself
+ * failed.
+ */
+int gqa_get_device_error(gqa_stream_t stream);
+
+/* A static English description of a status code. */
+const char *gqa_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int gqa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_ATTN_H */

@@ -1,0 +1,98 @@
+"""The C-ABI library loads, exports every entry point its header declares, and
+rejects bad arguments on the host before any CUDA call (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gqa_attention_forward_flash_b200 import binding
+from gqa_attention_forward_flash_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gqa_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return binding.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gqa_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("gqa_attention_fwd", "gqa_splitkv_combine", "gqa_attention_fwd_partial"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in binding.SIGNATURES, name
+
+
+def test_exported_symbols_are_c_linkage():
+    out = os.popen("nm -D --defined-only %s" % binding.LIB_PATH).read()
+    for name in declared_functions():
+        assert re.search(r"\bT %s$" % name, out, flags=re.M), name
+
+
+def test_version_and_status_strings(lib):
+    assert lib.gqa_version() >= 100
+    for code in binding.STATUS:
+        assert lib.gqa_status_string(code)
+
+
+P = ctypes.c_void_p
+
+
+def fwd(lib, q=16, k=16, v=16, kv=None, sink=None, out=16, lse=16, B=1, Hq=4, Hkv=1, Tq=4, Tkv=8, d=64,
+        scale=0.125, causal=0):
+    return lib.gqa_attention_fwd(P(q), P(k), P(v), P(kv), P(sink), P(out), P(lse), B, Hq, Hkv, Tq, Tkv, d,
+                                 scale, causal, None)
+
+
+def test_shape_errors(lib):
+    assert fwd(lib, Hq=6, Hkv=4) == -2          # Hq % Hkv
+    assert fwd(lib, Tkv=0) == -2                # no key buffer
+    assert fwd(lib, B=-1) == -2
+    assert fwd(lib, Hkv=0) == -2
+    assert fwd(lib, d=96) == -7                 # unsupported head dim
+    assert fwd(lib, B=1 << 20, Hq=1 << 10, Hkv=1 << 10, Tkv=1 << 12) == -2  # index overflow
+
+
+def test_null_and_alignment_errors(lib):
+    assert fwd(lib, q=0) == -1
+    assert fwd(lib, out=0) == -1
+    assert fwd(lib, k=24) == -3
+    assert fwd(lib, out=8) == -3
+
+
+def test_empty_problem_is_a_no_op(lib):
+    assert fwd(lib, B=0, q=0, k=0, v=0, out=0) == 0
+    assert fwd(lib, Tq=0, q=0, k=0, v=0, out=0) == 0
+
+
+def test_partial_and_combine_argument_errors(lib):
+    f = lib.gqa_attention_fwd_partial
+    assert f(P(16), P(16), P(16), None, 1, 4, 1, 4, 8, 64, 0.1, 0, 0, P(16), P(16), None) == -4
+    assert f(P(16), P(16), P(16), None, 1, 4, 1, 4, 8, 64, 0.1, 0, 257, P(16), P(16), None) == -4
+    assert f(P(16), P(16), P(16), None, 1, 4, 1, 4, 8, 64, 0.1, 0, 2, None, P(16), None) == -1
+    c = lib.gqa_splitkv_combine
+    assert c(P(16), P(16), 0, None, P(16), P(16), 1, 4, 4, 64, None) == -4
+    assert c(P(16), P(16), 2, None, P(16), P(16), 1, 4, 4, 66, None) == -2
+    assert c(None, P(16), 2, None, P(16), P(16), 1, 4, 4, 64, None) == -1
+    assert c(P(16), P(16), 2, None, P(24), P(16), 1, 4, 4, 64, None) == -3
+
+
+def test_valid_call_without_a_gpu_fails_loudly(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert fwd(lib) == -5  # GQA_ERR_CUDA: no silent CPU path

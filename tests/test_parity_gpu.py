@@ -1,0 +1,146 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small cases are compared element by element over the whole output; they span
+several key tiles, several q-tiles and ragged tails.  The full-size workloads
+are compared on sampled rows the oracle computes one by one, in the launch
+configuration the benchmark times.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gqa_attention_forward_flash_b200 import binding
+from gqa_attention_forward_flash_b200.synth import WORKLOADS, Workload, make_inputs, shrink
+
+from parity import compare, run_gpu, run_oracle, sample_rows, to_device
+
+pytestmark = pytest.mark.gpu
+
+W = WORKLOADS
+SMALL = {
+    "tiny_prefill": W["tiny_prefill"],
+    "decode_ragged_nan": shrink(W["batched_decode"], B=4, Tkv=1000),
+    "short_q_long_kv": shrink(W["short_q_long_kv"], B=2, Tkv=2000),
+    "causal_prefill_ragged": shrink(W["full_causal_prefill"], B=1, Hq=8, Hkv=2, Tq=700, Tkv=700),
+    "d64_causal_sink_ragged": Workload("d64", B=2, Hq=8, Hkv=2, Tq=37, Tkv=300, d=64, causal=True,
+                                       ragged=True, nan_pad=True, sink=True, seed=7),
+    "d256_sink_nan": Workload("d256", B=2, Hq=16, Hkv=2, Tq=3, Tkv=600, d=256, sigma=0.5, causal=True,
+                              sink=True, kv_len=555, nan_pad=True, seed=8),
+    "mha_g1": Workload("mha", B=2, Hq=4, Hkv=4, Tq=50, Tkv=260, d=128, seed=9),
+    "g32_two_qtiles": Workload("g32", B=1, Hq=32, Hkv=1, Tq=5, Tkv=400, d=128, causal=True, sink=True,
+                               seed=10),
+    "tq_gt_len_empty_rows": Workload("empty", B=2, Hq=4, Hkv=2, Tq=40, Tkv=64, d=128, causal=True,
+                                     kv_len=20, nan_pad=True, sink=True, seed=11),
+    "noncausal_prefill_d128": Workload("nc", B=1, Hq=8, Hkv=1, Tq=130, Tkv=515, d=128, seed=12),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_parity_small(name):
+    w = SMALL[name]
+    inp = make_inputs(w)
+    o, l = run_gpu(inp)
+    ro, rl = run_oracle(inp)
+    compare(o, l, ro, rl, name)
+
+
+def test_zero_and_full_lengths_with_sink():
+    w = Workload("zero", B=3, Hq=8, Hkv=2, Tq=4, Tkv=300, d=128, causal=True, sink=True, seed=13)
+    inp = make_inputs(w)
+    inp.kv_lens = torch.tensor([0, 300, 3], dtype=torch.int32)
+    inp.k[0] = float("nan")
+    inp.v[0] = float("nan")
+    o, l = run_gpu(inp)
+    ro, rl = run_oracle(inp)
+    compare(o, l, ro, rl, "zero-length batch")
+    # a batch with no key and a sink: O = 0 and lse = sink
+    assert np.all(o[0] == 0)
+    np.testing.assert_allclose(l[0], np.broadcast_to(inp.sink.numpy()[:, None], (8, 4)), atol=1e-6)
+
+
+def test_zero_length_without_sink_gives_minus_inf():
+    w = Workload("zero2", B=2, Hq=4, Hkv=1, Tq=2, Tkv=130, d=64, seed=14)
+    inp = make_inputs(w)
+    inp.kv_lens = torch.tensor([0, 130], dtype=torch.int32)
+    o, l = run_gpu(inp)
+    assert np.all(o[0] == 0) and np.all(np.isneginf(l[0]))
+    ro, rl = run_oracle(inp)
+    compare(o, l, ro, rl, "zero length")
+
+
+def test_constant_values_and_peaked_logits():
+    """|O| ~ 1 cases where max-abs is a meaningful bound: constant V rows return
+    that row; a query equal to a scaled key selects that key's value."""
+    w = Workload("const", B=2, Hq=8, Hkv=2, Tq=9, Tkv=700, d=128, causal=True, seed=15)
+    inp = make_inputs(w)
+    row = inp.v[0, 0, 0].clone()
+    inp.v[:] = row
+    o, l = run_gpu(inp)
+    np.testing.assert_allclose(o, np.broadcast_to(row.double().numpy(), o.shape), atol=8e-3, rtol=0)
+    inp2 = make_inputs(w)
+    inp2.q[:] = (inp2.k[:, :, 333:334, :].float().repeat_interleave(4, 1) * 3.0).to(torch.bfloat16)
+    o2, l2 = run_gpu(inp2)
+    ro2, rl2 = run_oracle(inp2)
+    compare(o2, l2, ro2, rl2, "peaked")
+    assert np.abs(ro2).max() > 0.5
+
+
+def test_deterministic_bitwise():
+    inp = make_inputs(SMALL["decode_ragged_nan"])
+    t = to_device(inp)
+    a, la = binding.gqa_attention_fwd(t["q"], t["k"], t["v"], t["kv_lens"], None, scale=inp.scale)
+    b, lb = binding.gqa_attention_fwd(t["q"], t["k"], t["v"], t["kv_lens"], None, scale=inp.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(la, lb)
+    assert binding.gqa_get_device_error() == 0
+
+
+@pytest.mark.parametrize("splits", [1, 3, 8])
+def test_forced_splits_then_combine(splits):
+    w = Workload("split", B=2, Hq=8, Hkv=2, Tq=3, Tkv=900, d=128, causal=True, sink=True, ragged=True,
+                 nan_pad=True, seed=16)
+    inp = make_inputs(w)
+    t = to_device(inp)
+    op, lp = binding.gqa_attention_fwd_partial(t["q"], t["k"], t["v"], t["kv_lens"], scale=inp.scale,
+                                               causal=True, num_splits=splits)
+    out, lse = binding.gqa_splitkv_combine(op, lp, t["sink"])
+    assert binding.gqa_get_device_error() == 0
+    ro, rl = run_oracle(inp)
+    compare(out.float().cpu().numpy(), lse.cpu().numpy(), ro, rl, "splits=%d" % splits)
+    # the oracle's own merge of the GPU partials agrees too
+    mo, ml = oracle.combine(op.cpu().numpy(), lp.cpu().numpy(), inp.sink)
+    compare(mo, ml, ro, rl, "oracle merge of GPU partials")
+
+
+def test_combine_kernel_on_oracle_partials():
+    """The public combine against the oracle's combine, on partials the oracle made."""
+    w = Workload("comb", B=2, Hq=4, Hkv=2, Tq=5, Tkv=64, d=128, causal=True, sink=True, seed=17)
+    inp = make_inputs(w)
+    cuts = [0, 7, 7, 30, 64]
+    parts = [oracle.attention_window(inp.q, inp.k, inp.v, None, None, inp.scale, True, a, b)
+             for a, b in zip(cuts[:-1], cuts[1:])]
+    po = np.stack([p[0] for p in parts], 3).astype(np.float32)
+    pl = np.stack([p[1] for p in parts], 3).astype(np.float32)
+    out, lse = binding.gqa_splitkv_combine(torch.from_numpy(po).cuda(), torch.from_numpy(pl).cuda(),
+                                           inp.sink.cuda())
+    mo, ml = oracle.combine(po, pl, inp.sink)
+    compare(out.float().cpu().numpy(), lse.cpu().numpy(), mo, ml, "combine")
+
+
+# ------------------------------------------------------------------ full size, sampled rows
+
+FULL = ["batched_decode", "short_q_long_kv", "full_causal_prefill"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_parity_full_size_sampled(name):
+    w = W[name]
+    inp = make_inputs(w)
+    o, l = run_gpu(inp)
+    assert np.all(np.isfinite(o))
+    rows = sample_rows(w.B, w.Hq, w.Tq, 384, seed=1)
+    ro, rl = oracle.attention_rows(inp.q, inp.k, inp.v, inp.kv_lens, inp.sink, inp.scale, inp.causal, rows)
+    compare(o.reshape(-1, w.d)[rows], l.reshape(-1)[rows], ro, rl, name)
