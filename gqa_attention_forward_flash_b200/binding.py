@@ -28,6 +28,8 @@ SIGNATURES = {
     "gqa_attention_fwd_partial": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P, _P]),
     "gqa_splitkv_combine": (_I, [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
     "gqa_get_device_error": (_I, [_P]),
+    "gqa_profile_begin": (_I, []),
+    "gqa_profile_take": (_I, [_P, _P, _I, _P]),
     "gqa_status_string": (ctypes.c_char_p, [_I]),
     "gqa_version": (_I, []),
 }
@@ -134,6 +136,19 @@ def gqa_splitkv_combine(o_part, lse_part, sink=None, out=None, lse=None, stream=
 
 def gqa_get_device_error(stream=None) -> int:
     return load().gqa_get_device_error(_stream(stream))
+
+
+def gqa_profile_begin() -> None:
+    _check("gqa_profile_begin", load().gqa_profile_begin())
+
+
+def gqa_profile_take(max_calls: int = 4096):
+    """Per-call (main kernel ms, combine kernel ms) since gqa_profile_begin."""
+    main = (ctypes.c_float * max_calls)()
+    comb = (ctypes.c_float * max_calls)()
+    n = ctypes.c_int(0)
+    _check("gqa_profile_take", load().gqa_profile_take(main, comb, max_calls, ctypes.byref(n)))
+    return list(main[:n.value]), list(comb[:n.value])
 
 
 def gqa_status_string(status: int) -> str:

@@ -36,6 +36,19 @@ struct DeviceState {
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
+
+// Optional per-launch timing (gqa_profile_*): events recorded on the launch
+// stream around the main kernel and around the combine kernel of each
+// gqa_attention_fwd call, read back by gqa_profile_take.
+constexpr int kProfCap = 4096;
+struct Prof {
+    bool on = false;
+    int dev = -1;
+    int n = 0;
+    cudaEvent_t ev[kProfCap][3];
+    bool created = false;
+};
+Prof g_prof;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 int get_state(DeviceState** out) {
@@ -247,9 +260,20 @@ extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, co
     p.meta = reinterpret_cast<long long*>(base + slot_o + slot_l);
     p.err = s->err;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaEvent_t* ev = nullptr;
+    if (g_prof.on && g_prof.n < kProfCap) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev == g_prof.dev) ev = g_prof.ev[g_prof.n++];
+    }
+    if (ev && cudaEventRecord(ev[0], st) != cudaSuccess) return GQA_ERR_CUDA;
     rc = dispatch_fwd(p, q, k, v, NC, st);
     if (rc) return rc;
-    return dispatch_combine_streamk(p, NC, st);
+    if (ev && cudaEventRecord(ev[1], st) != cudaSuccess) return GQA_ERR_CUDA;
+    rc = dispatch_combine_streamk(p, NC, st);
+    if (rc) return rc;
+    if (ev && cudaEventRecord(ev[2], st) != cudaSuccess) return GQA_ERR_CUDA;
+    return GQA_OK;
 }
 
 extern "C" int gqa_attention_fwd_partial(const void* q, const void* k, const void* v, const int32_t* kv_lens,
@@ -299,6 +323,45 @@ extern "C" int gqa_splitkv_combine(const float* o_part, const float* lse_part, i
     gqa_combine_uniform_kernel<<<static_cast<int>(blocks), 256, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
         o_part, lse_part, num_splits, sink, reinterpret_cast<__nv_bfloat16*>(out), lse, rows, Hq, Tq, d);
     return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+extern "C" int gqa_profile_begin(void) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
+    if (g_prof.created && g_prof.dev != dev) {
+        for (auto& e : g_prof.ev)
+            for (auto& x : e) cudaEventDestroy(x);
+        g_prof.created = false;
+    }
+    if (!g_prof.created) {
+        for (auto& e : g_prof.ev)
+            for (auto& x : e)
+                if (cudaEventCreate(&x) != cudaSuccess) return GQA_ERR_CUDA;
+        g_prof.created = true;
+    }
+    g_prof.dev = dev;
+    g_prof.n = 0;
+    g_prof.on = true;
+    return GQA_OK;
+}
+
+extern "C" int gqa_profile_take(float* main_ms, float* combine_ms, int max_calls, int* n_calls) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!n_calls) return GQA_ERR_NULL;
+    g_prof.on = false;
+    const int n = g_prof.n < max_calls ? g_prof.n : max_calls;
+    for (int i = 0; i < n; ++i) {
+        if (cudaEventSynchronize(g_prof.ev[i][2]) != cudaSuccess) return GQA_ERR_CUDA;
+        float a = 0.f, b = 0.f;
+        if (cudaEventElapsedTime(&a, g_prof.ev[i][0], g_prof.ev[i][1]) != cudaSuccess) return GQA_ERR_CUDA;
+        if (cudaEventElapsedTime(&b, g_prof.ev[i][1], g_prof.ev[i][2]) != cudaSuccess) return GQA_ERR_CUDA;
+        if (main_ms) main_ms[i] = a;
+        if (combine_ms) combine_ms[i] = b;
+    }
+    *n_calls = n;
+    g_prof.n = 0;
+    return GQA_OK;
 }
 
 extern "C" int gqa_get_device_error(gqa_stream_t stream) {
