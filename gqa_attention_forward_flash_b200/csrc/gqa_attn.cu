@@ -16,7 +16,7 @@
 #include <mutex>
 
 #include "gqa_attn.h"
-#include "gqa_fwd_kernel.cuh"
+#include "gqa_fwd2_kernel.cuh"
 
 namespace gqa {
 namespace {
@@ -30,8 +30,10 @@ struct DeviceState {
     int cc_major = 0, cc_minor = 0;
     long long clock_khz = 0;
     int* err = nullptr;          // device error word
-    void* scratch = nullptr;     // stream-K slots + meta
+    void* scratch = nullptr;     // stream-K partial slots (O, lse)
     size_t scratch_bytes = 0;
+    int* counters = nullptr;     // per-row-block merge tickets, all zero between calls
+    long long counters_len = 0;
 };
 
 std::mutex g_mu;
@@ -94,8 +96,10 @@ int make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int check_common(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int Tq, int Tkv, int d) {
+int check_common(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int Tq, int Tkv, int d,
+                 float scale) {
     if (B < 0 || Tq < 0 || Hq <= 0 || Hkv <= 0 || Tkv < 1) return GQA_ERR_SHAPE;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return GQA_ERR_SHAPE;
     if (Hq % Hkv != 0) return GQA_ERR_SHAPE;
     if (d != 64 && d != 128 && d != 256 && d != 512) return GQA_ERR_UNSUPPORTED;
     const long long qrows = static_cast<long long>(B) * Hq * Tq;
@@ -120,7 +124,9 @@ void fill_params(Params& p, int B, int Hq, int Hkv, int Tq, int Tkv, int d, floa
     p.R = p.G * Tq;
     p.QT = (p.R + BM - 1) / BM;
     p.U = B * Hkv;
-    p.W = static_cast<long long>(p.U) * p.QT;
+    p.RBQ = 1;
+    p.QW = p.QT;
+    p.W = static_cast<long long>(p.U) * p.QW;
     p.causal = causal ? 1 : 0;
     p.BN = BN;
     p.scale_log2 = scale * LOG2E;
@@ -131,20 +137,43 @@ void fill_params(Params& p, int B, int Hq, int Hkv, int Tq, int Tkv, int d, floa
     p.timeout_cycles = timeout;
 }
 
-// Kernel configurations per head dim (shared memory budget in FwdCfg).
-using Cfg64 = FwdCfg<64, 128, 4, 2>;
-using Cfg128 = FwdCfg<128, 128, 2, 2>;
-using Cfg256 = FwdCfg<256, 64, 2, 1>;
+// Kernel configurations (shared-memory and TMEM budgets are checked in the Cfg
+// structs).  Head dims 64 and 128 use the two-lane kernel: split-key lanes when
+// a unit's packed rows fit one 128-row q-tile (decode, short-q), dual-Q lanes
+// (two q-tiles per row-block sharing every K/V tile) otherwise.  Head dim 256
+// keeps one O accumulator (256 TMEM columns) and uses the single-lane kernel.
+using C2_64_SK = Fwd2Cfg<64, 4, 4, 1>;
+using C2_64_DQ = Fwd2Cfg<64, 4, 4, 2>;
+using C2_128_SK = Fwd2Cfg<128, 3, 3, 1>;
+using C2_128_DQ = Fwd2Cfg<128, 3, 2, 2>;
+using Cfg256 = FwdCfg<256, 64, 3, 2, 1>;
 
-template <class C>
-int launch_fwd(const Params& p0, const void* q, const void* k, const void* v, int grid, cudaStream_t stream) {
+// Tile geometry of the kernel that will serve these sizes.
+void choose_geometry(Params& p) {
+    if (p.d == 256) {
+        p.BN = Cfg256::BN;
+        p.RBQ = 1;
+    } else {
+        p.BN = 128;
+        p.RBQ = (p.R <= BM) ? 1 : 2;
+    }
+    p.QW = (p.QT + p.RBQ - 1) / p.RBQ;
+    p.W = static_cast<long long>(p.U) * p.QW;
+}
+
+template <class C, bool TWO_LANE>
+int launch_fwd(const Params& p0, const void* q, const void* k, const void* v, int grid, cudaStream_t stream,
+               cudaEvent_t ev_before, cudaEvent_t ev_after) {
     static bool attr_done[kMaxDevices] = {};
     int dev = 0;
-    cudaGetDevice(&dev);
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
     if (!attr_done[dev]) {
-        if (cudaFuncSetAttribute(gqa_fwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-            cudaSuccess)
-            return GQA_ERR_CUDA;
+        cudaError_t e;
+        if constexpr (TWO_LANE)
+            e = cudaFuncSetAttribute(gqa_fwd2_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        else
+            e = cudaFuncSetAttribute(gqa_fwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        if (e != cudaSuccess) return GQA_ERR_CUDA;
         attr_done[dev] = true;
     }
     CUtensorMap tq, tk, tv;
@@ -154,7 +183,11 @@ int launch_fwd(const Params& p0, const void* q, const void* k, const void* v, in
     // kernel zeroes in V and masks in S)
     const uint64_t qrows = static_cast<uint64_t>(p.B) * p.Hq * p.Tq;
     const uint64_t kvrows = static_cast<uint64_t>(p.B) * p.Hkv * p.Tkv;
-    p.q_box_rows = qrows < static_cast<uint64_t>(BM) ? static_cast<int>(qrows) : BM;
+    // few packed rows (decode): spread them over the four TMEM lane quadrants so
+    // that every SM sub-partition takes a share of the softmax
+    p.spread = (p.QT == 1 && p.R <= 96) ? 1 : 0;
+    p.rq = (p.R + 3) / 4;
+    p.q_box_rows = p.spread ? p.rq : (qrows < static_cast<uint64_t>(BM) ? static_cast<int>(qrows) : BM);
     p.kv_box_rows = kvrows < static_cast<uint64_t>(C::BN) ? static_cast<int>(kvrows) : C::BN;
     int rc = make_tmap(&tq, q, qrows, C::D, p.q_box_rows);
     if (rc) return rc;
@@ -162,36 +195,28 @@ int launch_fwd(const Params& p0, const void* q, const void* k, const void* v, in
     if (rc) return rc;
     rc = make_tmap(&tv, v, kvrows, C::D, p.kv_box_rows);
     if (rc) return rc;
-    gqa_fwd_kernel<C><<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
-    return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+    if (ev_before && cudaEventRecord(ev_before, stream) != cudaSuccess) return GQA_ERR_CUDA;
+    if constexpr (TWO_LANE)
+        gqa_fwd2_kernel<C><<<grid, NUM_THREADS2, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    else
+        gqa_fwd_kernel<C><<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+    if (ev_after && cudaEventRecord(ev_after, stream) != cudaSuccess) return GQA_ERR_CUDA;
+    return GQA_OK;
 }
 
-int bn_for(int d) {
-    switch (d) {
-        case 64: return Cfg64::BN;
-        case 128: return Cfg128::BN;
-        case 256: return Cfg256::BN;
-        default: return 0;
-    }
-}
-
-int dispatch_fwd(const Params& p, const void* q, const void* k, const void* v, int grid, cudaStream_t stream) {
+int dispatch_fwd(const Params& p, const void* q, const void* k, const void* v, int grid, cudaStream_t stream,
+                 cudaEvent_t e0 = nullptr, cudaEvent_t e1 = nullptr) {
     switch (p.d) {
-        case 64: return launch_fwd<Cfg64>(p, q, k, v, grid, stream);
-        case 128: return launch_fwd<Cfg128>(p, q, k, v, grid, stream);
-        case 256: return launch_fwd<Cfg256>(p, q, k, v, grid, stream);
+        case 64:
+            return p.RBQ == 1 ? launch_fwd<C2_64_SK, true>(p, q, k, v, grid, stream, e0, e1)
+                              : launch_fwd<C2_64_DQ, true>(p, q, k, v, grid, stream, e0, e1);
+        case 128:
+            return p.RBQ == 1 ? launch_fwd<C2_128_SK, true>(p, q, k, v, grid, stream, e0, e1)
+                              : launch_fwd<C2_128_DQ, true>(p, q, k, v, grid, stream, e0, e1);
+        case 256: return launch_fwd<Cfg256, false>(p, q, k, v, grid, stream, e0, e1);
         default: return GQA_ERR_UNSUPPORTED;
     }
-}
-
-int dispatch_combine_streamk(const Params& p, int grid, cudaStream_t stream) {
-    switch (p.d) {
-        case 64: gqa_combine_streamk_kernel<64><<<grid, 256, 0, stream>>>(p); break;
-        case 128: gqa_combine_streamk_kernel<128><<<grid, 256, 0, stream>>>(p); break;
-        case 256: gqa_combine_streamk_kernel<256><<<grid, 256, 0, stream>>>(p); break;
-        default: return GQA_ERR_UNSUPPORTED;
-    }
-    return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
 long long timeout_cycles(const DeviceState& s) {
@@ -202,6 +227,21 @@ long long timeout_cycles(const DeviceState& s) {
         if (v > 0) ms = v;
     }
     return s.clock_khz * ms;
+}
+
+int ensure_counters(DeviceState& s, long long n) {
+    if (s.counters_len >= n) return GQA_OK;
+    if (s.counters) {
+        if (cudaDeviceSynchronize() != cudaSuccess) return GQA_ERR_CUDA;
+        cudaFree(s.counters);
+        s.counters = nullptr;
+        s.counters_len = 0;
+    }
+    long long len = n < 4096 ? 4096 : n;
+    if (cudaMalloc(&s.counters, sizeof(int) * static_cast<size_t>(len)) != cudaSuccess) return GQA_ERR_CUDA;
+    if (cudaMemset(s.counters, 0, sizeof(int) * static_cast<size_t>(len)) != cudaSuccess) return GQA_ERR_CUDA;
+    s.counters_len = len;
+    return GQA_OK;
 }
 
 int ensure_scratch(DeviceState& s, size_t bytes) {
@@ -226,7 +266,7 @@ using namespace gqa;
 extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, const int32_t* kv_lens,
                                  const float* sink, void* out, float* lse, int B, int Hq, int Hkv, int Tq,
                                  int Tkv, int d, float scale, int causal, gqa_stream_t stream) {
-    int rc = check_common(q, k, v, B, Hq, Hkv, Tq, Tkv, d);
+    int rc = check_common(q, k, v, B, Hq, Hkv, Tq, Tkv, d, scale);
     if (rc) return rc;
     if (B == 0 || Tq == 0) return GQA_OK;
     if (!out) return GQA_ERR_NULL;
@@ -238,26 +278,29 @@ extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, co
     if (rc) return rc;
     if (s->cc_major != 10) return GQA_ERR_UNSUPPORTED;
     Params p;
-    fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale, causal, kv_lens, sink, out, lse, bn_for(d), timeout_cycles(*s));
+    fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale, causal, kv_lens, sink, out, lse, 0, timeout_cycles(*s));
+    choose_geometry(p);
     // grid: one CTA per SM; with host-known lengths never more CTAs than tiles
     int NC = s->sm_count < kMaxCtas ? s->sm_count : kMaxCtas;
     if (!kv_lens) {
         long long tot = 0;
-        for (int qt = 0; qt < p.QT; ++qt) tot += qtile_ntiles(p, qt, Tkv);
+        for (int qw = 0; qw < p.QW; ++qw) tot += qtile_ntiles(p, qw, Tkv);
         tot *= p.U;
         if (tot < NC) NC = static_cast<int>(tot);
     }
     if (NC < 1) NC = 1;
-    const size_t slot_o = static_cast<size_t>(2 * NC) * BM * d * sizeof(float);
-    const size_t slot_l = static_cast<size_t>(2 * NC) * BM * sizeof(float);
-    const size_t meta = static_cast<size_t>(NC) * 4 * sizeof(long long);
-    rc = ensure_scratch(*s, slot_o + slot_l + meta);
+    const size_t slot_rows = static_cast<size_t>(2 * NC) * BM * p.RBQ;
+    const size_t slot_o = slot_rows * d * sizeof(float);
+    const size_t slot_l = slot_rows * sizeof(float);
+    rc = ensure_scratch(*s, slot_o + slot_l);
+    if (rc) return rc;
+    rc = ensure_counters(*s, p.W);
     if (rc) return rc;
     char* base = static_cast<char*>(s->scratch);
     p.mode = 0;
     p.part_o = reinterpret_cast<float*>(base);
     p.part_lse = reinterpret_cast<float*>(base + slot_o);
-    p.meta = reinterpret_cast<long long*>(base + slot_o + slot_l);
+    p.counters = s->counters;
     p.err = s->err;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaEvent_t* ev = nullptr;
@@ -266,11 +309,7 @@ extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, co
         cudaGetDevice(&dev);
         if (dev == g_prof.dev) ev = g_prof.ev[g_prof.n++];
     }
-    if (ev && cudaEventRecord(ev[0], st) != cudaSuccess) return GQA_ERR_CUDA;
-    rc = dispatch_fwd(p, q, k, v, NC, st);
-    if (rc) return rc;
-    if (ev && cudaEventRecord(ev[1], st) != cudaSuccess) return GQA_ERR_CUDA;
-    rc = dispatch_combine_streamk(p, NC, st);
+    rc = dispatch_fwd(p, q, k, v, NC, st, ev ? ev[0] : nullptr, ev ? ev[1] : nullptr);
     if (rc) return rc;
     if (ev && cudaEventRecord(ev[2], st) != cudaSuccess) return GQA_ERR_CUDA;
     return GQA_OK;
@@ -279,7 +318,7 @@ extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, co
 extern "C" int gqa_attention_fwd_partial(const void* q, const void* k, const void* v, const int32_t* kv_lens,
                                          int B, int Hq, int Hkv, int Tq, int Tkv, int d, float scale, int causal,
                                          int num_splits, float* o_part, float* lse_part, gqa_stream_t stream) {
-    int rc = check_common(q, k, v, B, Hq, Hkv, Tq, Tkv, d);
+    int rc = check_common(q, k, v, B, Hq, Hkv, Tq, Tkv, d, scale);
     if (rc) return rc;
     if (num_splits < 1 || num_splits > GQA_MAX_SPLITS) return GQA_ERR_SPLITS;
     if (B == 0 || Tq == 0) return GQA_OK;
@@ -292,8 +331,9 @@ extern "C" int gqa_attention_fwd_partial(const void* q, const void* k, const voi
     if (rc) return rc;
     if (s->cc_major != 10) return GQA_ERR_UNSUPPORTED;
     Params p;
-    fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale, causal, kv_lens, nullptr, nullptr, nullptr, bn_for(d),
+    fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale, causal, kv_lens, nullptr, nullptr, nullptr, 0,
                 timeout_cycles(*s));
+    choose_geometry(p);
     const long long grid = p.W * num_splits;
     if (grid >= (1ll << 31)) return GQA_ERR_SHAPE;
     p.mode = 1;
@@ -372,7 +412,12 @@ extern "C" int gqa_get_device_error(gqa_stream_t stream) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return GQA_ERR_CUDA;
     int v = 0;
     if (cudaMemcpy(&v, s->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GQA_ERR_CUDA;
-    if (v != 0 && cudaMemset(s->err, 0, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
+    if (v != 0) {
+        if (cudaMemset(s->err, 0, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
+        // an aborted launch may leave merge tickets behind
+        if (s->counters && cudaMemset(s->counters, 0, sizeof(int) * static_cast<size_t>(s->counters_len)) != cudaSuccess)
+            return GQA_ERR_CUDA;
+    }
     return v;
 }
 

@@ -4,14 +4,24 @@
 // BM = 128 "packed" query rows: the G query heads that share the KV head times
 // their Tq rows (AstrAI commit log, head-packing commit: K/V tiles stream once
 // per block instead of once per q head).  Roles:
-//   warp 0      TMA producer: Q tile per segment, ring of K and V tiles
-//   warp 1      TMEM owner and single-thread tcgen05 MMA issuer:
-//                 S = Q K^T into one of two TMEM S buffers,
-//                 O += P V into the TMEM O accumulator
-//   warps 2..5  softmax / correction / epilogue, one packed row per thread:
-//                 logical-length + causal mask by selection, online (m, l)
-//                 carry with lazy rescale of O, P -> bf16 into shared memory,
-//                 final O / l (or a normalised partial + lse) to global memory
+//   warp 0 lane 0   TMA producer of the Q tile (per segment) and the K ring
+//   warp 0 lane 16  TMA producer of the V ring (so a K prefetch never waits
+//                   for a V stage to drain)
+//   warp 1          TMEM owner; lane 0 issues every tcgen05 MMA:
+//                     S = Q K^T   (A, B from shared memory) into TMEM S[g % 2]
+//                     O += P V    (A = P from TMEM, B = V from shared memory)
+//   warps 2..9      softmax / correction / epilogue: warp w reads TMEM lane
+//                     quadrant w % 4 (one packed row per thread) and half
+//                     (w - 2) / 4 of every S tile's columns (its exponentials and
+//                     its half of O); each reads the whole S row for the row max,
+//                     so the two warps of a sub-partition never wait for each
+//                     other inside the key loop.  Logical-
+//                     length + causal mask by selection, online (m, l) carry with
+//                     a lazy rescale of O, P -> bf16 into TMEM P[g % 2], final
+//                     O / l (or a normalised partial + lse) to global memory.
+//                   With few packed rows (decode) the Q tile is loaded as four
+//                   short boxes, one per lane quadrant, so that all four SM
+//                   sub-partitions share the softmax work.
 // (nvfp4-megamoe-kernel dsv4/kernels/attention commit log: multi-tile commit for
 // the online softmax over KV tiles, prefill commits for the TMEM row/lane
 // mapping, epilogue commits for TMEM -> registers -> global.)
@@ -20,10 +30,12 @@
 // range of nkv(w) tiles of BN keys.  All tiles of all row-blocks are laid out
 // in one flat order and cut into NC equal contiguous spans, one per CTA
 // ("stream-K"): every CTA gets the same number of tiles whatever the lengths.
-// A row-block finished inside one CTA is written straight to `out`; one cut by
-// span boundaries leaves normalised fp32 partials in per-CTA slots, merged by
-// the LSE combine kernel (AstrAI commit log: split-KV scratch commit;
-// kernbench2 benches commit log: associative (m, l, O) merge).
+// A row-block finished inside one CTA is written straight to `out`.  One cut by
+// span boundaries leaves normalised fp32 partials (O, lse) in per-CTA slots;
+// each contributing CTA then takes a ticket on the row-block's counter and the
+// last one merges all partials with the LSE combine and writes `out` (AstrAI
+// commit log: split-KV scratch commit, and the last-block fold with an atomic
+// ticket and fences; kernbench2 benches commit log: associative (m, l, O) merge).
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda.h>
@@ -34,7 +46,9 @@
 namespace gqa {
 
 constexpr int BM = 128;          // packed query rows per tile = TMEM lanes
-constexpr int NUM_THREADS = 192; // 6 warps
+constexpr int NUM_THREADS = 320; // 10 warps: producers, MMA, 8 softmax warps (2 per lane quadrant)
+constexpr int NSOFT = 256;       // softmax threads
+constexpr int NSOFT_WARPS = NSOFT / 32;  // arrivals per softmax-side barrier phase (one per warp)
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
@@ -46,22 +60,26 @@ constexpr int DEV_ERR_KVLEN = -8;
 struct Params {
     int B, Hq, Hkv, Tq, Tkv, d;
     int G, R, QT, U;      // R = G*Tq rows per unit, QT = ceil(R/BM) q-tiles, U = B*Hkv units
-    long long W;          // row-blocks = U*QT
+    int RBQ;              // q-tiles per row-block (1, or 2 when two q-tiles share every K/V tile)
+    int QW;               // row-blocks per unit = ceil(QT / RBQ)
+    long long W;          // row-blocks = U*QW
     int causal;
-    int BN;               // keys per tile (set by the launcher to the kernel's BN)
-    float scale_log2;     // scale * log2(e)
+    int BN;               // keys per tile (the kernel's BN)
+    float scale_log2;     // scale * log2(e)  (> 0)
     const int* kv_lens;   // [B] or null
     const float* sink;    // [Hq] or null
     __nv_bfloat16* out;   // [B,Hq,Tq,d]
     float* lse;           // [B,Hq,Tq] or null
-    int mode;             // 0: stream-K (direct + slots); 1: uniform splits (partials only)
+    int mode;             // 0: stream-K (direct + slots + in-kernel merge); 1: uniform splits
     int num_splits;       // mode 1
     float* part_o;        // mode 0: [2*NC][BM][d] slots; mode 1: [B,Hq,Tq,S,d]
     float* part_lse;      // mode 0: [2*NC][BM];      mode 1: [B,Hq,Tq,S]
-    long long* meta;      // mode 0: [NC][4] per-CTA combine record
+    int* counters;        // mode 0: [W] merge tickets, zero between calls
     int* err;             // device error word
     long long timeout_cycles;
-    int q_box_rows;       // rows of one Q TMA box: min(BM, B*Hq*Tq)
+    int q_box_rows;       // rows of one Q TMA box: min(BM, B*Hq*Tq), or rq in the spread layout
+    int spread;           // 1: packed row r lives in TMEM lane (r / rq) * 32 + r % rq (R <= 96)
+    int rq;               // packed rows per lane quadrant in the spread layout
     int kv_box_rows;      // rows of one K/V TMA box: min(BN, B*Hkv*Tkv)
 };
 
@@ -84,10 +102,17 @@ __host__ __device__ inline int qtile_extent(const Params& p, int qt, int n) {
     return ext < 0 ? 0 : ext;
 }
 
-// Tiles of a row-block; at least one, so that a row-block with no visible key
-// is still visited (its one tile is fully masked and it writes O = 0).
-__host__ __device__ inline int qtile_ntiles(const Params& p, int qt, int n) {
-    const int ext = qtile_extent(p, qt, n);
+// Key tiles of row-block wq of a unit (its q-tiles wq*RBQ ...), at least one, so
+// that a row-block with no visible key is still visited (its one tile is fully
+// masked and it writes O = 0).
+__host__ __device__ inline int qtile_ntiles(const Params& p, int wq, int n) {
+    int ext = 0;
+    const int q0 = wq * p.RBQ;
+    const int q1 = (q0 + p.RBQ < p.QT) ? q0 + p.RBQ : p.QT;
+    for (int qt = q0; qt < q1; ++qt) {
+        const int e = qtile_extent(p, qt, n);
+        ext = e > ext ? e : ext;
+    }
     const int t = (ext + p.BN - 1) / p.BN;
     return t < 1 ? 1 : t;
 }
@@ -101,12 +126,13 @@ __host__ __device__ inline long long span_begin(int c, long long tot, int NC) {
 }
 
 struct Seg {
-    int w;        // row-block (< 2^31 is checked on the host)
-    int t0, t1;   // tile range inside the row-block
-    int ntiles;   // nkv(w)
-    int n;        // logical length of the row-block's batch
-    int kind;     // 0: direct, 1: stream-K slot, 2: uniform split
-    int slot;     // slot (kind 1) or split index (kind 2)
+    int w;          // row-block
+    int t0, t1;     // tile range inside the row-block
+    int ntiles;     // nkv(w)
+    int n;          // logical length of the row-block's batch
+    int kind;       // 0: direct, 1: stream-K slot, 2: uniform split
+    int slot;       // slot (kind 1) or split index (kind 2)
+    long long pw;   // flat index of the row-block's first tile (kind 0/1)
 };
 
 __device__ __forceinline__ int load_len(const Params& p, int b) {
@@ -127,11 +153,11 @@ __device__ __forceinline__ long long warp_sum_ll(long long v) {
 __device__ long long unit_tiles_warp(const Params& p, int n) {
     if (!p.causal) {
         int t = (n + p.BN - 1) / p.BN;
-        return static_cast<long long>(p.QT) * (t < 1 ? 1 : t);
+        return static_cast<long long>(p.QW) * (t < 1 ? 1 : t);
     }
     const int lane = threadIdx.x & 31;
     long long acc = 0;
-    for (int qt = lane; qt < p.QT; qt += 32) acc += qtile_ntiles(p, qt, n);
+    for (int qt = lane; qt < p.QW; qt += 32) acc += qtile_ntiles(p, qt, n);
     return warp_sum_ll(acc);
 }
 
@@ -152,7 +178,6 @@ __device__ void plan_span(const Params& p, int c, int NC, SpanStart* out) {
     const long long p0 = span_begin(c, tot, NC), p1 = span_begin(c + 1, tot, NC);
     int w = 0, t = 0;
     if (p0 < p1) {
-        // batch, then unit, then q-tile containing flat index p0
         long long acc = 0;
         int b = 0, n = p.Tkv;
         long long per_unit = 0;
@@ -179,10 +204,9 @@ __device__ void plan_span(const Params& p, int c, int NC, SpanStart* out) {
             qt = static_cast<int>(rem / nt);
             rem -= static_cast<long long>(qt) * nt;
         } else {
-            // warp scan over q-tiles, 32 at a time
-            for (int base = 0; base < p.QT; base += 32) {
+            for (int base = 0; base < p.QW; base += 32) {
                 const int q = base + lane;
-                long long cnt = q < p.QT ? qtile_ntiles(p, q, n) : 0;
+                long long cnt = q < p.QW ? qtile_ntiles(p, q, n) : 0;
                 long long inc = cnt;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -201,7 +225,7 @@ __device__ void plan_span(const Params& p, int c, int NC, SpanStart* out) {
                 rem -= chunk_total;
             }
         }
-        w = u * p.QT + qt;
+        w = u * p.QW + qt;
         t = static_cast<int>(rem);
     }
     if (lane == 0) {
@@ -213,24 +237,41 @@ __device__ void plan_span(const Params& p, int c, int NC, SpanStart* out) {
     }
 }
 
-// Walks this CTA's segments (every role keeps its own copy; all see the same sequence).
+// Walks this CTA's segments; every role keeps its own walker and all see the
+// same sequence.  Mode 1 has exactly one (possibly empty) segment per CTA.
 struct SegWalker {
     int w, t;
-    long long remaining;
-    bool first;
+    long long remaining, pos;
+    bool first, single_done;
     int c;
 
-    __device__ void init_streamk(const SpanStart& s, int cta) {
+    __device__ void init(const Params& p, const SpanStart& s, int cta) {
         w = s.w;
         t = s.t;
-        remaining = s.p1 - s.p0;
+        remaining = (p.mode == 0) ? s.p1 - s.p0 : 0;
+        pos = s.p0;
         first = true;
+        single_done = (p.mode == 0);
         c = cta;
     }
-    // mode 0
     __device__ bool next(const Params& p, Seg& sg) {
+        if (!single_done) {  // mode 1: CTA = (row-block, split)
+            single_done = true;
+            const int S = p.num_splits;
+            sg.w = c / S;
+            const int s = c % S;
+            const int u = sg.w / p.QW, qt = sg.w % p.QW;
+            sg.n = load_len(p, u / p.Hkv);
+            sg.ntiles = qtile_ntiles(p, qt, sg.n);
+            sg.t0 = static_cast<int>((static_cast<long long>(s) * sg.ntiles) / S);
+            sg.t1 = static_cast<int>((static_cast<long long>(s + 1) * sg.ntiles) / S);
+            sg.kind = 2;
+            sg.slot = s;
+            sg.pw = 0;
+            return true;
+        }
         if (remaining <= 0) return false;
-        const int u = w / p.QT, qt = w % p.QT;
+        const int u = w / p.QW, qt = w % p.QW;
         const int n = load_len(p, u / p.Hkv);
         const int nt = qtile_ntiles(p, qt, n);
         long long take = nt - t;
@@ -240,9 +281,10 @@ struct SegWalker {
         sg.t1 = t + static_cast<int>(take);
         sg.ntiles = nt;
         sg.n = n;
-        const bool full = (t == 0 && sg.t1 == nt);
-        sg.kind = full ? 0 : 1;
+        sg.kind = (t == 0 && sg.t1 == nt) ? 0 : 1;
         sg.slot = first ? 2 * c : 2 * c + 1;
+        sg.pw = pos - t;
+        pos += take;
         remaining -= take;
         first = false;
         ++w;
@@ -251,25 +293,11 @@ struct SegWalker {
     }
 };
 
-// mode 1: CTA = (row-block, split); the single segment may be empty (t0 == t1).
-__device__ inline void uniform_segment(const Params& p, int cta, Seg& sg) {
-    const int S = p.num_splits;
-    sg.w = cta / S;
-    const int s = cta % S;
-    const int u = sg.w / p.QT, qt = sg.w % p.QT;
-    sg.n = load_len(p, u / p.Hkv);
-    sg.ntiles = qtile_ntiles(p, qt, sg.n);
-    sg.t0 = static_cast<int>((static_cast<long long>(s) * sg.ntiles) / S);
-    sg.t1 = static_cast<int>((static_cast<long long>(s + 1) * sg.ntiles) / S);
-    sg.kind = 2;
-    sg.slot = s;
-}
-
 // ------------------------------------------------------------------ kernel config
 
-template <int D_, int BN_, int ST_, int QBUF_>
+template <int D_, int BN_, int STK_, int STV_, int QBUF_>
 struct FwdCfg {
-    static constexpr int D = D_, BN = BN_, ST = ST_, QBUF = QBUF_;
+    static constexpr int D = D_, BN = BN_, STK = STK_, STV = STV_, QBUF = QBUF_;
     static_assert(D % 64 == 0 && D <= 256, "head dim");
     static_assert(BN == 64 || BN == 128, "key tile");
     static constexpr int NBOX = D / 64;                 // 64-column swizzle boxes per row
@@ -277,35 +305,35 @@ struct FwdCfg {
     static constexpr int Q_BYTES = NBOX * Q_BOX;
     static constexpr int KV_BOX = BN * 128;
     static constexpr int KV_BYTES = NBOX * KV_BOX;      // one K (or V) tile
-    static constexpr int P_BOX = BM * 128;
-    static constexpr int P_BYTES = (BN / 64) * P_BOX;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + QBUF * Q_BYTES;
-    static constexpr int OFF_V = OFF_K + ST * KV_BYTES;
-    static constexpr int OFF_P = OFF_V + ST * KV_BYTES;
-    static constexpr int OFF_BAR = OFF_P + P_BYTES;
+    static constexpr int OFF_V = OFF_K + STK * KV_BYTES;
+    static constexpr int OFF_BAR = OFF_V + STV * KV_BYTES;
     // barrier indices
     static constexpr int B_QFULL = 0;
     static constexpr int B_QEMPTY = B_QFULL + QBUF;
     static constexpr int B_KFULL = B_QEMPTY + QBUF;
-    static constexpr int B_KEMPTY = B_KFULL + ST;
-    static constexpr int B_VFULL = B_KEMPTY + ST;
-    static constexpr int B_VEMPTY = B_VFULL + ST;
-    static constexpr int B_SFULL = B_VEMPTY + ST;   // 2
-    static constexpr int B_SFREE = B_SFULL + 2;     // 2
-    static constexpr int B_PFULL = B_SFREE + 2;
-    static constexpr int B_ODONE = B_PFULL + 1;
-    static constexpr int B_FINAL = B_ODONE + 1;
-    static constexpr int NBAR = B_FINAL + 1;
+    static constexpr int B_KEMPTY = B_KFULL + STK;
+    static constexpr int B_VFULL = B_KEMPTY + STK;
+    static constexpr int B_VEMPTY = B_VFULL + STV;
+    static constexpr int B_SFULL = B_VEMPTY + STV;  // [2]
+    static constexpr int B_SFREE = B_SFULL + 2;     // [2]
+    static constexpr int B_PFULL = B_SFREE + 2;     // [2]
+    static constexpr int B_ODONE = B_PFULL + 2;     // [2]
+    static constexpr int B_FINAL = B_ODONE + 2;
+    static constexpr int B_XSYNC = B_FINAL + 1;     // softmax-group barrier (bounded waits, abort-safe)
+    static constexpr int NBAR = B_XSYNC + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr int MISC_BYTES = 64;
+    static constexpr int MISC_BYTES = 1664;
     static constexpr int SMEM_USED = OFF_MISC + MISC_BYTES;
     static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack to align the base to 1024
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-    // TMEM columns
+    // TMEM columns: O [0, D), S[2] of BN fp32 columns, P[2] of BN/2 columns (bf16 pairs)
     static constexpr uint32_t TM_O = 0;
-    static constexpr uint32_t TM_S0 = 256;
+    static constexpr uint32_t TM_S = D;
+    static constexpr uint32_t TM_P = D + 2 * BN;
     static constexpr uint32_t TM_COLS = 512;
+    static_assert(D + 3 * BN <= 512, "TMEM budget");
     static constexpr uint32_t IDESC_S = ptx::umma_idesc_bf16_f32(BM, BN, false, false);
     static constexpr uint32_t IDESC_PV = ptx::umma_idesc_bf16_f32(BM, D, false, true);
 };
@@ -313,10 +341,12 @@ struct FwdCfg {
 struct Misc {
     uint32_t tmem_base;
     volatile int abort;
-    int pad0, pad1;
-    SpanStart span;   // 40 bytes
+    volatile int merge_flag;
+    int pad;
+    SpanStart span;     // 40 bytes
+    float red[2][BM];   // per-half row maxima / row sums, by TMEM lane
+    float mlse[BM];     // merged lse per packed row (in-kernel merge)
 };
-static_assert(sizeof(Misc) <= 64, "misc block");
 
 // Bounded wait; on expiry records GQA_ERR_TIMEOUT and raises the CTA abort flag.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Misc* misc, const Params& p) {
@@ -330,6 +360,14 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Misc* mi
             misc->abort = 1;
             return false;
         }
+    }
+}
+// Bounded drain used at teardown (no abort short-cut: copies must land).
+__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t issued, long long limit) {
+    if (issued == 0) return;
+    const uint32_t par = (issued - 1) & 1;
+    const long long t0 = clock64();
+    while (!ptx::mbar_try_wait(bar, par) && clock64() - t0 < limit) {
     }
 }
 
@@ -347,16 +385,23 @@ struct RB {
 };
 __device__ __forceinline__ RB rb_of(const Params& p, int w) {
     RB r;
-    const int u = w / p.QT;
-    r.qt = w % p.QT;
+    const int u = w / p.QW;
+    r.qt = (w % p.QW) * p.RBQ;  // first q-tile of the row-block
     r.b = u / p.Hkv;
     r.g = u % p.Hkv;
     r.q_row0 = (static_cast<long long>(r.b) * p.Hq + static_cast<long long>(r.g) * p.G) * p.Tq +
                static_cast<long long>(r.qt) * BM;
     r.kv_row0 = static_cast<long long>(u) * p.Tkv;
     const int left = p.R - r.qt * BM;
-    r.rows_valid = left < BM ? left : BM;
+    r.rows_valid = left < BM * p.RBQ ? left : BM * p.RBQ;
     return r;
+}
+
+// Slot a contributing CTA wrote for row-block (flat start pw): its first segment
+// (2c) unless it is the CTA that holds the row-block's first tile inside a span
+// that began earlier (then its last segment, 2c + 1).
+__device__ __forceinline__ long long merge_slot(int cc, int c_first, bool c0_first) {
+    return (cc == c_first && !c0_first) ? 2ll * cc + 1 : 2ll * cc;
 }
 
 template <class C>
@@ -382,20 +427,29 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ptx::mbar_init(bar(C::B_QFULL + i), 1);
             ptx::mbar_init(bar(C::B_QEMPTY + i), 1);
         }
-        for (int i = 0; i < C::ST; ++i) {
+        for (int i = 0; i < C::STK; ++i) {
             ptx::mbar_init(bar(C::B_KFULL + i), 1);
             ptx::mbar_init(bar(C::B_KEMPTY + i), 1);
+        }
+        for (int i = 0; i < C::STV; ++i) {
             ptx::mbar_init(bar(C::B_VFULL + i), 1);
             ptx::mbar_init(bar(C::B_VEMPTY + i), 1);
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(bar(C::B_SFULL + i), 1);
-            ptx::mbar_init(bar(C::B_SFREE + i), 128);
+            ptx::mbar_init(bar(C::B_SFREE + i), NSOFT_WARPS);
+            ptx::mbar_init(bar(C::B_PFULL + i), NSOFT_WARPS);
+            ptx::mbar_init(bar(C::B_ODONE + i), 1);
         }
-        ptx::mbar_init(bar(C::B_PFULL), 128);
-        ptx::mbar_init(bar(C::B_ODONE), 1);
         ptx::mbar_init(bar(C::B_FINAL), 1);
+        ptx::mbar_init(bar(C::B_XSYNC), NSOFT_WARPS);
         misc->abort = 0;
+        misc->merge_flag = 0;
+        if (p.mode != 0) {
+            misc->span.tot = 0;
+            misc->span.p0 = misc->span.p1 = 0;
+            misc->span.w = misc->span.t = 0;
+        }
         ptx::fence_mbar_init();
         ptx::tma_prefetch_desc(&tm_q);
         ptx::tma_prefetch_desc(&tm_k);
@@ -411,150 +465,120 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     ptx::tc_fence_after();
     const uint32_t tmem = misc->tmem_base;
 
-    // ---------------------------------------------------------------- producer
+    // ---------------------------------------------------------------- producers
     if (warp == 0) {
         if (lane == 0) {
+            // Q tile per segment + K ring
             const uint64_t pol_q = ptx::policy_evict_last();
             const uint64_t pol_kv = (p.QT == 1) ? ptx::policy_evict_first() : ptx::policy_evict_normal();
             SegWalker wk;
+            wk.init(p, misc->span, cta);
             Seg sg;
-            bool more;
-            if (p.mode == 0) wk.init_streamk(misc->span, cta);
             int seg_i = 0;
             uint32_t g = 0;
             bool ok = true;
-            bool single_done = false;
-            uint32_t k_issued[C::ST], v_issued[C::ST], q_issued[C::QBUF];
-            for (int i = 0; i < C::ST; ++i) k_issued[i] = v_issued[i] = 0;
+            uint32_t k_issued[C::STK], q_issued[C::QBUF];
+            for (int i = 0; i < C::STK; ++i) k_issued[i] = 0;
             for (int i = 0; i < C::QBUF; ++i) q_issued[i] = 0;
-            while (ok) {
-                if (p.mode == 0) {
-                    more = wk.next(p, sg);
-                } else {
-                    more = !single_done;
-                    single_done = true;
-                    if (more) uniform_segment(p, cta, sg);
-                }
-                if (!more) break;
+            while (ok && wk.next(p, sg)) {
                 if (sg.t1 <= sg.t0) continue;  // empty split: nothing to load
                 const RB rb = rb_of(p, sg.w);
                 const int qb = seg_i % C::QBUF;
                 ok = wait_bar(bar(C::B_QEMPTY + qb), ((seg_i / C::QBUF) & 1) ^ 1, misc, p);
                 if (!ok) break;
-                ptx::mbar_arrive_expect_tx(bar(C::B_QFULL + qb), C::NBOX * p.q_box_rows * 128);
+                const int nq = p.spread ? 4 : 1;
+                ptx::mbar_arrive_expect_tx(bar(C::B_QFULL + qb), nq * C::NBOX * p.q_box_rows * 128);
                 ++q_issued[qb];
-                for (int bx = 0; bx < C::NBOX; ++bx)
-                    ptx::tma_load_2d(sbase + C::OFF_Q + qb * C::Q_BYTES + bx * C::Q_BOX, &tm_q, bx * 64,
-                                     static_cast<int>(rb.q_row0), bar(C::B_QFULL + qb), pol_q);
-                for (int t = sg.t0; t < sg.t1 && ok; ++t, ++g) {
-                    const int st = g % C::ST;
-                    const uint32_t ph = ((g / C::ST) & 1) ^ 1;
-                    const int y = static_cast<int>(rb.kv_row0 + static_cast<long long>(t) * C::BN);
-                    ok = wait_bar(bar(C::B_KEMPTY + st), ph, misc, p);
+                for (int qq = 0; qq < nq; ++qq)
+                    for (int bx = 0; bx < C::NBOX; ++bx)
+                        ptx::tma_load_2d(sbase + C::OFF_Q + qb * C::Q_BYTES + bx * C::Q_BOX + qq * 32 * 128, &tm_q,
+                                         bx * 64, static_cast<int>(rb.q_row0) + qq * p.rq, bar(C::B_QFULL + qb),
+                                         pol_q);
+                for (int t = sg.t0; t < sg.t1; ++t, ++g) {
+                    const int st = g % C::STK;
+                    ok = wait_bar(bar(C::B_KEMPTY + st), ((g / C::STK) & 1) ^ 1, misc, p);
                     if (!ok) break;
+                    const int y = static_cast<int>(rb.kv_row0 + static_cast<long long>(t) * C::BN);
                     ptx::mbar_arrive_expect_tx(bar(C::B_KFULL + st), C::NBOX * p.kv_box_rows * 128);
                     ++k_issued[st];
                     for (int bx = 0; bx < C::NBOX; ++bx)
-                        ptx::tma_load_2d(sbase + C::OFF_K + st * C::KV_BYTES + bx * C::KV_BOX, &tm_k,
-                                         bx * 64, y, bar(C::B_KFULL + st), pol_kv);
-                    ok = wait_bar(bar(C::B_VEMPTY + st), ph, misc, p);
-                    if (!ok) break;
-                    ptx::mbar_arrive_expect_tx(bar(C::B_VFULL + st), C::NBOX * p.kv_box_rows * 128);
-                    ++v_issued[st];
-                    for (int bx = 0; bx < C::NBOX; ++bx)
-                        ptx::tma_load_2d(sbase + C::OFF_V + st * C::KV_BYTES + bx * C::KV_BOX, &tm_v,
-                                         bx * 64, y, bar(C::B_VFULL + st), pol_kv);
+                        ptx::tma_load_2d(sbase + C::OFF_K + st * C::KV_BYTES + bx * C::KV_BOX, &tm_k, bx * 64, y,
+                                         bar(C::B_KFULL + st), pol_kv);
                 }
                 ++seg_i;
             }
-            // Never leave the CTA with copies in flight: wait (bounded) for the last
-            // load issued into every stage and Q buffer, also after an abort.
-            auto drain = [&](uint32_t b, uint32_t issued) {
-                if (issued == 0) return;
-                const uint32_t par = (issued - 1) & 1;
-                const long long t0 = clock64();
-                while (!ptx::mbar_try_wait(b, par) && clock64() - t0 < p.timeout_cycles) {}
-            };
-            for (int i = 0; i < C::ST; ++i) {
-                drain(bar(C::B_KFULL + i), k_issued[i]);
-                drain(bar(C::B_VFULL + i), v_issued[i]);
-            }
-            for (int i = 0; i < C::QBUF; ++i) drain(bar(C::B_QFULL + i), q_issued[i]);
-        } else if (lane == 1 && p.mode == 0) {
-            // Per-CTA combine record: this CTA starts a row-block it does not finish.
-            const SpanStart s = misc->span;
-            long long rec[4] = {-1, 0, 0, s.tot};
-            if (s.p1 > s.p0) {
-                SegWalker wk;
-                wk.init_streamk(s, cta);
-                Seg sg, last;
-                int count = 0;
-                while (wk.next(p, sg)) { last = sg; ++count; }
-                if (count > 0 && last.t0 == 0 && last.t1 < last.ntiles) {
-                    const long long pw = s.p1 - (last.t1 - last.t0);
-                    rec[0] = last.w;
-                    rec[1] = cta_of(pw + last.ntiles - 1, s.tot, NC);
-                    rec[2] = last.slot;
+            // never leave the CTA with copies in flight
+            for (int i = 0; i < C::STK; ++i) drain_bar(bar(C::B_KFULL + i), k_issued[i], p.timeout_cycles);
+            for (int i = 0; i < C::QBUF; ++i) drain_bar(bar(C::B_QFULL + i), q_issued[i], p.timeout_cycles);
+        } else if (lane == 16) {
+            // V ring
+            const uint64_t pol_kv = (p.QT == 1) ? ptx::policy_evict_first() : ptx::policy_evict_normal();
+            SegWalker wk;
+            wk.init(p, misc->span, cta);
+            Seg sg;
+            uint32_t g = 0;
+            bool ok = true;
+            uint32_t v_issued[C::STV];
+            for (int i = 0; i < C::STV; ++i) v_issued[i] = 0;
+            while (ok && wk.next(p, sg)) {
+                if (sg.t1 <= sg.t0) continue;
+                const RB rb = rb_of(p, sg.w);
+                for (int t = sg.t0; t < sg.t1; ++t, ++g) {
+                    const int st = g % C::STV;
+                    ok = wait_bar(bar(C::B_VEMPTY + st), ((g / C::STV) & 1) ^ 1, misc, p);
+                    if (!ok) break;
+                    const int y = static_cast<int>(rb.kv_row0 + static_cast<long long>(t) * C::BN);
+                    ptx::mbar_arrive_expect_tx(bar(C::B_VFULL + st), C::NBOX * p.kv_box_rows * 128);
+                    ++v_issued[st];
+                    for (int bx = 0; bx < C::NBOX; ++bx)
+                        ptx::tma_load_2d(sbase + C::OFF_V + st * C::KV_BYTES + bx * C::KV_BOX, &tm_v, bx * 64, y,
+                                         bar(C::B_VFULL + st), pol_kv);
                 }
             }
-            long long* m = p.meta + 4ll * cta;
-            m[0] = rec[0];
-            m[1] = rec[1];
-            m[2] = rec[2];
-            m[3] = rec[3];
+            for (int i = 0; i < C::STV; ++i) drain_bar(bar(C::B_VFULL + i), v_issued[i], p.timeout_cycles);
         }
     }
     // ---------------------------------------------------------------- MMA issuer
     else if (warp == 1) {
         if (lane == 0) {
             SegWalker wk;
+            wk.init(p, misc->span, cta);
             Seg sg;
-            bool more;
-            if (p.mode == 0) wk.init_streamk(misc->span, cta);
             int seg_i = 0;
             uint32_t g = 0;
             bool ok = true;
-            bool single_done = false;
-            bool have_prev = false;     // a PV is pending for tile g-1
-            bool prev_first = false;    // ... and it is the first tile of its segment
+            bool have_prev = false;   // a PV is pending for tile g-1
+            bool prev_first = false;  // ... and it is the first tile of its segment
             const uint32_t tm_o = tmem + C::TM_O;
 
             auto issue_pv = [&](uint32_t gp, bool first_of_seg) -> bool {
-                if (!wait_bar(bar(C::B_PFULL), gp & 1, misc, p)) return false;
-                const int st = gp % C::ST;
-                if (!wait_bar(bar(C::B_VFULL + st), (gp / C::ST) & 1, misc, p)) return false;
+                const int pb = gp & 1;
+                if (!wait_bar(bar(C::B_PFULL + pb), (gp >> 1) & 1, misc, p)) return false;
+                const int st = gp % C::STV;
+                if (!wait_bar(bar(C::B_VFULL + st), (gp / C::STV) & 1, misc, p)) return false;
                 ptx::tc_fence_after();
-                const uint32_t pbase = sbase + C::OFF_P;
                 const uint32_t vbase = sbase + C::OFF_V + st * C::KV_BYTES;
+                const uint32_t tm_p = tmem + C::TM_P + pb * (C::BN / 2);
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk) {
-                    const uint64_t ad = ptx::umma_desc_sw128(pbase + (kk >> 2) * C::P_BOX + (kk & 3) * 32, 16, 1024);
                     const uint64_t bd = ptx::umma_desc_sw128(vbase + kk * 2048, C::KV_BOX, 1024);
-                    ptx::umma_bf16_ss(tm_o, ad, bd, C::IDESC_PV, (kk > 0 || !first_of_seg) ? 1u : 0u);
+                    ptx::umma_bf16_ts(tm_o, tm_p + kk * 8, bd, C::IDESC_PV, (kk > 0 || !first_of_seg) ? 1u : 0u);
                 }
-                ptx::umma_commit(bar(C::B_ODONE));
+                ptx::umma_commit(bar(C::B_ODONE + pb));
                 ptx::umma_commit(bar(C::B_VEMPTY + st));
                 return true;
             };
 
-            while (ok) {
-                if (p.mode == 0) {
-                    more = wk.next(p, sg);
-                } else {
-                    more = !single_done;
-                    single_done = true;
-                    if (more) uniform_segment(p, cta, sg);
-                }
-                if (!more) break;
+            while (ok && wk.next(p, sg)) {
                 if (sg.t1 <= sg.t0) continue;
                 const int qb = seg_i % C::QBUF;
                 ok = wait_bar(bar(C::B_QFULL + qb), (seg_i / C::QBUF) & 1, misc, p);
                 if (!ok) break;
                 const uint32_t qbase = sbase + C::OFF_Q + qb * C::Q_BYTES;
                 for (int t = sg.t0; t < sg.t1; ++t, ++g) {
-                    const int st = g % C::ST;
+                    const int st = g % C::STK;
                     const int sb = g & 1;
-                    ok = wait_bar(bar(C::B_KFULL + st), (g / C::ST) & 1, misc, p);
+                    ok = wait_bar(bar(C::B_KFULL + st), (g / C::STK) & 1, misc, p);
                     if (!ok) break;
                     if (g >= 2) {
                         ok = wait_bar(bar(C::B_SFREE + sb), ((g >> 1) - 1) & 1, misc, p);
@@ -562,7 +586,7 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     }
                     ptx::tc_fence_after();
                     const uint32_t kbase = sbase + C::OFF_K + st * C::KV_BYTES;
-                    const uint32_t tm_s = tmem + C::TM_S0 + sb * 128;
+                    const uint32_t tm_s = tmem + C::TM_S + sb * C::BN;
 #pragma unroll
                     for (int kk = 0; kk < C::D / 16; ++kk) {
                         const uint32_t off = (kk & 3) * 32;
@@ -583,48 +607,61 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 ++seg_i;
             }
             if (ok && have_prev) ok = issue_pv(g - 1, prev_first);
-            // make sure every MMA has retired before TMEM is released
+            // every MMA must retire before TMEM is released
             ptx::umma_commit(bar(C::B_FINAL));
-            const long long t0 = clock64();
-            while (!ptx::mbar_try_wait(bar(C::B_FINAL), 0) && clock64() - t0 < p.timeout_cycles) {}
+            drain_bar(bar(C::B_FINAL), 1, p.timeout_cycles);
         }
     }
     // ---------------------------------------------------------------- softmax / epilogue
     else {
-        const int quad = warp & 3;
-        const int row = quad * 32 + lane;
+        const int quad = warp & 3;             // TMEM lane quadrant this warp may access
+        const int half = (warp - 2) >> 2;      // which half of the key columns / O columns
+        const int lrow = quad * 32 + lane;     // TMEM lane = row of the MMA tile
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-        const uint32_t tm_o = tmem + lane_off + C::TM_O;
+        constexpr int HB = C::BN / 2;          // key columns per half
+        constexpr int HD = C::D / 2;           // O columns per half
+        const uint32_t tm_o = tmem + lane_off + C::TM_O + half * HD;
+        const int stid = threadIdx.x - 64;     // 0..255 among the softmax threads
+        // Barrier over the 256 softmax threads on an mbarrier with a bounded wait, so
+        // that an abort elsewhere can never leave threads parked at it.
+        uint32_t xph = 0;
+        auto xsync = [&]() -> bool {
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(C::B_XSYNC));
+            const bool r = wait_bar(bar(C::B_XSYNC), xph & 1, misc, p);
+            ++xph;
+            return __all_sync(0xffffffffu, r);
+        };
         SegWalker wk;
+        wk.init(p, misc->span, cta);
         Seg sg;
-        bool more;
-        if (p.mode == 0) wk.init_streamk(misc->span, cta);
         uint32_t g = 0;
         bool ok = true;
-        bool single_done = false;
-        uint8_t* const p_smem = smem + C::OFF_P;
 
-        while (ok) {
-            if (p.mode == 0) {
-                more = wk.next(p, sg);
-            } else {
-                more = !single_done;
-                single_done = true;
-                if (more) uniform_segment(p, cta, sg);
-            }
-            if (!more) break;
+        while (ok && wk.next(p, sg)) {
             const RB rb = rb_of(p, sg.w);
-            const int rp = rb.qt * BM + row;           // packed row inside the unit
-            const bool valid = row < rb.rows_valid;
-            const int hl = valid ? rp / p.Tq : 0;      // head inside the group
+            // packed row held by this thread
+            int rloc;                           // row inside the q-tile
+            bool valid, active;
+            if (p.spread) {
+                rloc = quad * p.rq + lane;
+                valid = lane < p.rq && rloc < rb.rows_valid;
+                active = quad * p.rq < rb.rows_valid;
+            } else {
+                rloc = lrow;
+                valid = lrow < rb.rows_valid;
+                active = quad * 32 < rb.rows_valid;
+            }
+            const int rp = rb.qt * BM + rloc;   // packed row inside the unit
+            const int hl = valid ? rp / p.Tq : 0;
             const int i = valid ? rp % p.Tq : 0;
             int limit = p.causal ? (sg.n - p.Tq + i) : (sg.n - 1);
             if (limit > sg.n - 1) limit = sg.n - 1;
             if (!valid) limit = -1;
             const int h = rb.g * p.G + hl;
 
-            float m_ref = -INFINITY;  // log2-domain running max used for P
-            float l_sum = 0.f;
+            float m_ref = -INFINITY;  // log2-domain running max the P values are taken against
+            float l_sum = 0.f;        // this half's running sum
 
             for (int t = sg.t0; t < sg.t1; ++t, ++g) {
                 const int sb = g & 1;
@@ -632,179 +669,295 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 ptx::tc_fence_after();
-                float s[C::BN];
-                {
-                    const uint32_t tm_s = tmem + lane_off + C::TM_S0 + sb * 128;
+                float s[HB];
+                float mx = -INFINITY;
+                if (active) {
+                    const uint32_t tm_s = tmem + lane_off + C::TM_S + sb * C::BN;
+                    // own half: kept for the exponentials
 #pragma unroll
-                    for (int c = 0; c < C::BN / 32; ++c) {
+                    for (int c = 0; c < HB / 32; ++c) {
                         uint32_t r[32];
-                        ptx::tmem_ld32(tm_s + c * 32, r);
+                        ptx::tmem_ld32(tm_s + half * HB + c * 32, r);
 #pragma unroll
                         for (int j = 0; j < 32; ++j) s[c * 32 + j] = __uint_as_float(r[j]);
                     }
                     ptx::tmem_wait_ld();
+                    // mask by selection (never by adding -inf: NaN + -inf stays NaN)
+                    const int lim_all = limit - t * C::BN;      // last visible column of the tile
+                    const bool full = __all_sync(0xffffffffu, lim_all >= C::BN - 1);
+                    const int lim = lim_all - half * HB;
+                    if (!full) {
+#pragma unroll
+                        for (int c = 0; c < HB; ++c) s[c] = (c <= lim) ? s[c] : -INFINITY;
+                    }
+                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                    for (int c = 0; c < HB; c += 4) {
+                        m4[0] = fmaxf(m4[0], s[c]);
+                        m4[1] = fmaxf(m4[1], s[c + 1]);
+                        m4[2] = fmaxf(m4[2], s[c + 2]);
+                        m4[3] = fmaxf(m4[3], s[c + 3]);
+                    }
+                    // other half: only its maximum is needed
+                    const int olim = lim_all - (half ^ 1) * HB;
+#pragma unroll
+                    for (int c = 0; c < HB / 32; ++c) {
+                        uint32_t r[32];
+                        ptx::tmem_ld32(tm_s + (half ^ 1) * HB + c * 32, r);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float x = __uint_as_float(r[j + e]);
+                                m4[e] = fmaxf(m4[e], (full || c * 32 + j + e <= olim) ? x : -INFINITY);
+                            }
+                        }
+                    }
+                    mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
                 }
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(bar(C::B_SFREE + sb));
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar(C::B_SFREE + sb));
 
-                // mask (select, never add: NaN + -inf would stay NaN) and row max
-                const int lim = limit - t * C::BN;
-                float mx = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < C::BN; ++c) {
-                    const float x = (c <= lim) ? s[c] * p.scale_log2 : -INFINITY;
-                    s[c] = x;
-                    mx = fmaxf(mx, x);
-                }
                 const bool first = (t == sg.t0);
                 float alpha = 1.f;
+                const float mt = mx * p.scale_log2;  // -inf stays -inf (scale > 0)
                 if (first) {
-                    m_ref = mx;
-                } else if (mx > m_ref + RESCALE_THRESHOLD) {
-                    alpha = exp2f(m_ref - mx);
-                    m_ref = mx;
+                    m_ref = mt;
+                } else if (mt > m_ref + RESCALE_THRESHOLD) {
+                    alpha = ptx::ex2(m_ref - mt);
+                    m_ref = mt;
                 }
-                const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-
-                // the previous PV must be done: P buffer reuse and O rescale
-                if (g >= 1) {
-                    ok = wait_bar(bar(C::B_ODONE), (g - 1) & 1, misc, p);
+                // P buffer g%2 was last read by PV_{g-2}
+                const int pb = g & 1;
+                if (g >= 2) {
+                    ok = wait_bar(bar(C::B_ODONE + pb), ((g >> 1) - 1) & 1, misc, p);
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
                     ptx::tc_fence_after();
                 }
-                if (!first && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-                    for (int c = 0; c < C::D / 32; ++c) {
-                        uint32_t r[32];
-                        ptx::tmem_ld32(tm_o + c * 32, r);
-                        ptx::tmem_wait_ld();
+                if (active) {
+                    const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+                    const uint32_t tm_p = tmem + lane_off + C::TM_P + pb * (C::BN / 2) + half * (HB / 2);
+                    float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
-                        ptx::tmem_st32(tm_o + c * 32, r);
+                    for (int c = 0; c < HB / 32; ++c) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float a = ptx::ex2(fmaf(s[c * 32 + 2 * j], p.scale_log2, neg_m));
+                            const float b = ptx::ex2(fmaf(s[c * 32 + 2 * j + 1], p.scale_log2, neg_m));
+                            rs4[(2 * j) & 3] += a;
+                            rs4[(2 * j + 1) & 3] += b;
+                            pk[j] = pack_bf16x2(a, b);
+                        }
+                        ptx::tmem_st16(tm_p + c * 16, pk);
+                    }
+                    l_sum = l_sum * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
+                    // lazy rescale of this half of O: only when some row's max grew by more than 2^8
+                    if (!first && __any_sync(0xffffffffu, alpha != 1.f)) {
+                        bool okw = wait_bar(bar(C::B_ODONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, misc, p);
+                        okw = __all_sync(0xffffffffu, okw);
+                        if (!okw) {
+                            ok = false;
+                        } else {
+                            ptx::tc_fence_after();
+#pragma unroll 1
+                            for (int c = 0; c < HD / 32; ++c) {
+                                uint32_t r[32];
+                                ptx::tmem_ld32(tm_o + c * 32, r);
+                                ptx::tmem_wait_ld();
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
+                                ptx::tmem_st32(tm_o + c * 32, r);
+                            }
+                        }
                     }
                     ptx::tmem_wait_st();
                 }
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 // padded key rows of the V tile must reach the MMA as zeros (0 * NaN = NaN)
                 if ((t + 1) * C::BN > sg.n) {
-                    const int st = g % C::ST;
-                    ok = wait_bar(bar(C::B_VFULL + st), (g / C::ST) & 1, misc, p);
+                    const int st = g % C::STV;
+                    ok = wait_bar(bar(C::B_VFULL + st), (g / C::STV) & 1, misc, p);
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
                     int z0 = sg.n - t * C::BN;
                     z0 = z0 < 0 ? 0 : z0;
                     uint8_t* vt = smem + C::OFF_V + st * C::KV_BYTES;
                     const int chunks = (C::BN - z0) * C::NBOX * 8;  // 16-byte chunks
-                    for (int q = threadIdx.x - 64; q < chunks; q += 128) {
+                    for (int q = stid; q < chunks; q += NSOFT) {
                         const int r = z0 + q / (C::NBOX * 8);
                         const int rem = q % (C::NBOX * 8);
-                        const int bx = rem / 8, ch = rem % 8;
-                        *reinterpret_cast<uint4*>(vt + bx * C::KV_BOX + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4*>(vt + (rem >> 3) * C::KV_BOX + r * 128 + (rem & 7) * 16) =
+                            make_uint4(0, 0, 0, 0);
                     }
+                    ptx::fence_proxy_async_smem();
                 }
-                // P = exp2(x - m) -> bf16, written in the 128-byte-swizzled K-major image
-                float rs = 0.f;
-#pragma unroll
-                for (int c8 = 0; c8 < C::BN / 8; ++c8) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float a = exp2f(s[c8 * 8 + 2 * j] - m_use);
-                        const float b = exp2f(s[c8 * 8 + 2 * j + 1] - m_use);
-                        pk[j] = pack_bf16x2(a, b);
-                        rs += a + b;
-                    }
-                    const int bx = c8 >> 3;
-                    const int ch = (c8 & 7) ^ (row & 7);
-                    *reinterpret_cast<uint4*>(p_smem + bx * C::P_BOX + row * 128 + ch * 16) =
-                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                }
-                l_sum = l_sum * alpha + rs;
-                ptx::fence_proxy_async_smem();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(bar(C::B_PFULL));
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar(C::B_PFULL + pb));
             }
             if (!ok) break;
 
             // ------------------------------------------------ segment epilogue
-            float o_scale = 0.f, lse_v = -INFINITY;
-            if (sg.t1 > sg.t0) {
-                ok = wait_bar(bar(C::B_ODONE), (g - 1) & 1, misc, p);
+            const bool nonempty = sg.t1 > sg.t0;
+            misc->red[half][lrow] = l_sum;
+            if (!xsync()) { ok = false; break; }
+            const float l_tot = l_sum + misc->red[half ^ 1][lrow];
+            if (nonempty) {
+                const uint32_t gl = g - 1;
+                ok = wait_bar(bar(C::B_ODONE + (gl & 1)), (gl >> 1) & 1, misc, p);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 ptx::tc_fence_after();
+            }
+            float o_scale = 0.f, lse_v = -INFINITY;
+            if (nonempty) {
                 if (sg.kind == 0) {
                     const float sk = (p.sink != nullptr && valid) ? __ldg(p.sink + h) * LOG2E : -INFINITY;
                     const float M = fmaxf(m_ref, sk);
                     if (M != -INFINITY) {
-                        const float a = exp2f(m_ref - M);
-                        const float lt = l_sum * a + exp2f(sk - M);
+                        const float a = ptx::ex2(m_ref - M);
+                        const float lt = l_tot * a + ptx::ex2(sk - M);
                         o_scale = a / lt;
-                        lse_v = (M + log2f(lt)) * LN2;
+                        lse_v = (M + __log2f(lt)) * LN2;
                     }
-                } else if (l_sum > 0.f) {
-                    o_scale = 1.f / l_sum;
-                    lse_v = (m_ref + log2f(l_sum)) * LN2;
+                } else if (l_tot > 0.f) {
+                    o_scale = 1.f / l_tot;
+                    lse_v = (m_ref + __log2f(l_tot)) * LN2;
                 }
             }
-            // destination of this row
-            const long long fr = rb.q_row0 + row;  // flat row (b*Hq + h)*Tq + i when valid
+            const long long fr = rb.q_row0 + rloc;  // flat row (b*Hq + h)*Tq + i when valid
             if (sg.kind == 0) {
-                __nv_bfloat16* dst = p.out + fr * C::D;
+                __nv_bfloat16* dst = p.out + fr * C::D + half * HD;
+                if (active) {
 #pragma unroll 1
-                for (int c = 0; c < C::D / 32; ++c) {
-                    uint32_t r[32];
-                    if (sg.t1 > sg.t0) {
+                    for (int c = 0; c < HD / 32; ++c) {
+                        uint32_t r[32];
                         ptx::tmem_ld32(tm_o + c * 32, r);
                         ptx::tmem_wait_ld();
-                    }
-                    if (valid) {
-                        uint32_t pk[16];
+                        if (valid) {
+                            uint32_t pk[16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            pk[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * o_scale,
-                                                __uint_as_float(r[2 * j + 1]) * o_scale);
-                        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+                            for (int j = 0; j < 16; ++j)
+                                pk[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * o_scale,
+                                                    __uint_as_float(r[2 * j + 1]) * o_scale);
+                            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) d4[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                            for (int j = 0; j < 4; ++j)
+                                d4[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                        }
                     }
                 }
-                if (valid && p.lse != nullptr) p.lse[fr] = lse_v;
+                if (valid && half == 0 && p.lse != nullptr) p.lse[fr] = lse_v;
             } else {
                 float* dst;
                 float* dl;
                 if (sg.kind == 1) {
-                    dst = p.part_o + (static_cast<long long>(sg.slot) * BM + row) * C::D;
-                    dl = p.part_lse + static_cast<long long>(sg.slot) * BM + row;
+                    dst = p.part_o + (static_cast<long long>(sg.slot) * BM + rloc) * C::D + half * HD;
+                    dl = p.part_lse + static_cast<long long>(sg.slot) * BM + rloc;
                 } else {
-                    dst = p.part_o + (fr * p.num_splits + sg.slot) * C::D;
+                    dst = p.part_o + (fr * p.num_splits + sg.slot) * C::D + half * HD;
                     dl = p.part_lse + fr * p.num_splits + sg.slot;
                 }
+                if (active) {
 #pragma unroll 1
-                for (int c = 0; c < C::D / 32; ++c) {
-                    uint32_t r[32];
-                    if (sg.t1 > sg.t0) {
-                        ptx::tmem_ld32(tm_o + c * 32, r);
-                        ptx::tmem_wait_ld();
-                    }
-                    if (valid) {
-                        float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+                    for (int c = 0; c < HD / 32; ++c) {
+                        uint32_t r[32];
+                        if (nonempty) {
+                            ptx::tmem_ld32(tm_o + c * 32, r);
+                            ptx::tmem_wait_ld();
+                        }
+                        if (valid) {
+                            float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            float4 v4;
-                            if (sg.t1 > sg.t0) {
-                                v4 = make_float4(__uint_as_float(r[4 * j]) * o_scale, __uint_as_float(r[4 * j + 1]) * o_scale,
-                                                 __uint_as_float(r[4 * j + 2]) * o_scale, __uint_as_float(r[4 * j + 3]) * o_scale);
-                            } else {
-                                v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                            for (int j = 0; j < 8; ++j) {
+                                float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                                if (nonempty)
+                                    v4 = make_float4(__uint_as_float(r[4 * j]) * o_scale,
+                                                     __uint_as_float(r[4 * j + 1]) * o_scale,
+                                                     __uint_as_float(r[4 * j + 2]) * o_scale,
+                                                     __uint_as_float(r[4 * j + 3]) * o_scale);
+                                __stcg(d4 + j, v4);
                             }
-                            d4[j] = v4;
                         }
                     }
                 }
-                if (valid) *dl = lse_v;
+                if (valid && half == 0) __stcg(dl, lse_v);
+
+                if (sg.kind == 1) {
+                    __threadfence();  // this thread's partial rows are visible before the ticket
+                    // ---- ticket: the last CTA to finish a piece of this row-block merges
+                    const long long tot = misc->span.tot;
+                    const int c_first = cta_of(sg.pw, tot, NC);
+                    const int c_last = cta_of(sg.pw + sg.ntiles - 1, tot, NC);
+                    if (!xsync()) { ok = false; break; }
+                    if (stid == 0) {
+                        int ncontrib = 0;
+                        for (int cc = c_first; cc <= c_last; ++cc)
+                            ncontrib += span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC);
+                        __threadfence();
+                        const int old = atomicAdd(p.counters + sg.w, 1);
+                        const int last = (old == ncontrib - 1);
+                        if (last) __threadfence();
+                        misc->merge_flag = last;
+                    }
+                    if (!xsync()) { ok = false; break; }
+                    if (misc->merge_flag) {
+                        __threadfence();
+                        const bool c0_first = span_begin(c_first, tot, NC) == sg.pw;
+                        // merged lse per packed row
+                        for (int r = stid; r < rb.rows_valid; r += NSOFT) {
+                            const int hr = rb.g * p.G + (rb.qt * BM + r) / p.Tq;
+                            float L = (p.sink != nullptr) ? __ldg(p.sink + hr) : -INFINITY;
+                            for (int cc = c_first; cc <= c_last; ++cc) {
+                                if (!(span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC))) continue;
+                                L = fmaxf(L, __ldcg(p.part_lse + merge_slot(cc, c_first, c0_first) * BM + r));
+                            }
+                            float lt = -INFINITY;
+                            if (L != -INFINITY) {
+                                float z = (p.sink != nullptr) ? __expf(__ldg(p.sink + hr) - L) : 0.f;
+                                for (int cc = c_first; cc <= c_last; ++cc) {
+                                    if (!(span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC))) continue;
+                                    z += __expf(__ldcg(p.part_lse + merge_slot(cc, c_first, c0_first) * BM + r) - L);
+                                }
+                                lt = L + __logf(z);
+                            }
+                            misc->mlse[r] = lt;
+                            if (p.lse != nullptr) p.lse[rb.q_row0 + r] = lt;
+                        }
+                        if (!xsync()) { ok = false; break; }
+                        // weighted sum of the partials, 8 columns per item
+                        constexpr int C8 = C::D / 8;
+                        for (int it = stid; it < rb.rows_valid * C8; it += NSOFT) {
+                            const int r = it / C8, c8 = it % C8;
+                            const float lt = misc->mlse[r];
+                            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                            if (lt != -INFINITY) {
+                                for (int cc = c_first; cc <= c_last; ++cc) {
+                                    if (!(span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC))) continue;
+                                    const long long sl = merge_slot(cc, c_first, c0_first);
+                                    const float wgt = __expf(__ldcg(p.part_lse + sl * BM + r) - lt);
+                                    const float4* src =
+                                        reinterpret_cast<const float4*>(p.part_o + (sl * BM + r) * C::D + 8 * c8);
+                                    const float4 a = __ldcg(src), b = __ldcg(src + 1);
+                                    acc[0] += wgt * a.x; acc[1] += wgt * a.y; acc[2] += wgt * a.z; acc[3] += wgt * a.w;
+                                    acc[4] += wgt * b.x; acc[5] += wgt * b.y; acc[6] += wgt * b.z; acc[7] += wgt * b.w;
+                                }
+                            }
+                            *reinterpret_cast<uint4*>(p.out + (rb.q_row0 + r) * C::D + 8 * c8) =
+                                make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                           pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+                        }
+                        if (stid == 0) p.counters[sg.w] = 0;  // ready for the next call
+                    }
+                }
             }
             ptx::tc_fence_before();
+            // misc->red / mlse / merge_flag are reused by the next segment
+            if (!xsync()) { ok = false; break; }
         }
     }
 
@@ -817,74 +970,7 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
 }
 
-// ------------------------------------------------------------------ combine kernels
-
-// Stream-K combine: block c merges the row-block that CTA c started but did not finish.
-template <int D>
-__global__ void __launch_bounds__(256)
-gqa_combine_streamk_kernel(const Params p) {
-    const int c = blockIdx.x;
-    const int NC = gridDim.x;
-    const long long* m = p.meta + 4ll * c;
-    const long long w = m[0];
-    if (w < 0) return;
-    const int c_last = static_cast<int>(m[1]);
-    const int slot0 = static_cast<int>(m[2]);
-    const long long tot = m[3];
-    if (w >= p.W || c_last < c || c_last >= NC || slot0 < 0 || slot0 >= 2 * NC || tot <= 0) {
-        if (threadIdx.x == 0) atomicCAS(p.err, 0, DEV_ERR_TIMEOUT);
-        return;
-    }
-
-    __shared__ int slots[512];
-    __shared__ int nslots;
-    __shared__ float row_lse[BM];
-    if (threadIdx.x == 0) {
-        int k = 0;
-        slots[k++] = slot0;
-        for (int cc = c + 1; cc <= c_last && k < 512; ++cc)
-            if (span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC)) slots[k++] = 2 * cc;
-        nslots = k;
-    }
-    __syncthreads();
-    const int ns = nslots;
-    const RB rb = rb_of(p, static_cast<int>(w));
-    for (int r = threadIdx.x; r < rb.rows_valid; r += blockDim.x) {
-        const int rp = rb.qt * BM + r;
-        const int h = rb.g * p.G + rp / p.Tq;
-        float L = (p.sink != nullptr) ? __ldg(p.sink + h) : -INFINITY;
-        for (int k = 0; k < ns; ++k) L = fmaxf(L, p.part_lse[static_cast<long long>(slots[k]) * BM + r]);
-        float lt = -INFINITY;
-        if (L != -INFINITY) {
-            float z = (p.sink != nullptr) ? __expf(__ldg(p.sink + h) - L) : 0.f;
-            for (int k = 0; k < ns; ++k) z += __expf(p.part_lse[static_cast<long long>(slots[k]) * BM + r] - L);
-            lt = L + __logf(z);
-        }
-        row_lse[r] = lt;
-        if (p.lse != nullptr) p.lse[rb.q_row0 + r] = lt;
-    }
-    __syncthreads();
-    constexpr int C4 = D / 4;
-    for (int it = threadIdx.x; it < rb.rows_valid * C4; it += blockDim.x) {
-        const int r = it / C4, c4 = it % C4;
-        const float lt = row_lse[r];
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (lt != -INFINITY) {
-            for (int k = 0; k < ns; ++k) {
-                const long long sl = slots[k];
-                const float wgt = __expf(p.part_lse[sl * BM + r] - lt);
-                if (wgt == 0.f) continue;
-                const float4 o = *reinterpret_cast<const float4*>(p.part_o + (sl * BM + r) * D + 4 * c4);
-                acc.x += wgt * o.x;
-                acc.y += wgt * o.y;
-                acc.z += wgt * o.z;
-                acc.w += wgt * o.w;
-            }
-        }
-        uint2 pk = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
-        *reinterpret_cast<uint2*>(p.out + (rb.q_row0 + r) * D + 4 * c4) = pk;
-    }
-}
+// ------------------------------------------------------------------ public combine kernel
 
 // Uniform combine (public entry): one warp per row, S partials laid out [rows, S, d].
 __global__ void __launch_bounds__(256)
@@ -933,3 +1019,5 @@ gqa_combine_uniform_kernel(const float* __restrict__ o_part, const float* __rest
 }
 
 }  // namespace gqa
+
+static_assert(sizeof(gqa::Misc) <= 1664, "misc block");

@@ -64,6 +64,9 @@ def test_shape_errors(lib):
     assert fwd(lib, B=-1) == -2
     assert fwd(lib, Hkv=0) == -2
     assert fwd(lib, d=96) == -7                 # unsupported head dim
+    assert fwd(lib, scale=0.0) == -2            # the scale must be positive and finite
+    assert fwd(lib, scale=-1.0) == -2
+    assert fwd(lib, scale=float("inf")) == -2
     assert fwd(lib, B=1 << 20, Hq=1 << 10, Hkv=1 << 10, Tkv=1 << 12) == -2  # index overflow
 
 

@@ -88,6 +88,35 @@ def test_constant_values_and_peaked_logits():
     assert np.abs(ro2).max() > 0.5
 
 
+def _ramped(seed, Tkv=4000):
+    """Keys whose norm grows along the sequence, so that the running row max
+    grows tile after tile and the lazy O rescale has to fire."""
+    w = Workload("ramp", B=2, Hq=8, Hkv=2, Tq=3, Tkv=Tkv, d=128, causal=True, sink=True, seed=seed)
+    inp = make_inputs(w)
+    ramp = torch.linspace(0.1, 6.0, Tkv).view(1, 1, Tkv, 1)
+    inp.k = (inp.k.float() * ramp).to(torch.bfloat16)
+    return inp
+
+
+def test_rescale_path_stream_split():
+    inp = _ramped(18)
+    o, l = run_gpu(inp)
+    ro, rl = run_oracle(inp)
+    compare(o, l, ro, rl, "ramped keys")
+
+
+def test_rescale_path_single_cta_per_row_block():
+    """num_splits = 1: one CTA walks all key tiles of a row-block."""
+    inp = _ramped(19, Tkv=6000)
+    t = to_device(inp)
+    op, lp = binding.gqa_attention_fwd_partial(t["q"], t["k"], t["v"], None, scale=inp.scale, causal=True,
+                                               num_splits=1)
+    out, lse = binding.gqa_splitkv_combine(op, lp, t["sink"])
+    assert binding.gqa_get_device_error() == 0
+    ro, rl = run_oracle(inp)
+    compare(out.float().cpu().numpy(), lse.cpu().numpy(), ro, rl, "one split, ramped keys")
+
+
 def test_deterministic_bitwise():
     inp = make_inputs(SMALL["decode_ragged_nan"])
     t = to_device(inp)
