@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libgqa_attn.so")
 STATUS = {
     0: "GQA_OK", -1: "GQA_ERR_NULL", -2: "GQA_ERR_SHAPE", -3: "GQA_ERR_ALIGN", -4: "GQA_ERR_SPLITS",
     -5: "GQA_ERR_CUDA", -6: "GQA_ERR_TIMEOUT", -7: "GQA_ERR_UNSUPPORTED", -8: "GQA_ERR_KVLEN",
+    -9: "GQA_ERR_SCRATCH",
 }
 MAX_SPLITS = 256
 
@@ -25,6 +26,7 @@ MAX_SPLITS = 256
 _P, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 SIGNATURES = {
     "gqa_attention_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "gqa_attention_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "gqa_attention_fwd_partial": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P, _P]),
     "gqa_splitkv_combine": (_I, [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
     "gqa_get_device_error": (_I, [_P]),
@@ -100,6 +102,28 @@ def gqa_attention_fwd(q, k, v, kv_lens=None, sink=None, out=None, lse=None, scal
     rc = load().gqa_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_lens), _ptr(sink), _ptr(out), _ptr(lse),
                                   B, Hq, Hkv, Tq, Tkv, d, float(scale), int(bool(causal)), _stream(stream))
     _check("gqa_attention_fwd", rc)
+    return out, lse
+
+
+def gqa_attention_fwd_noalloc(q, k, v, kv_lens=None, sink=None, out=None, lse=None, scale=None, causal=False,
+                              stream=None):
+    """gqa_attention_fwd without device allocation inside the library (its split
+    scratch is a fixed array in the library; see include/gqa_attn.h)."""
+    _need(q, torch.bfloat16, "q", 4)
+    _need(k, torch.bfloat16, "k", 4)
+    _need(v, torch.bfloat16, "v", 4)
+    B, Hq, Tq, d = q.shape
+    _, Hkv, Tkv, _ = k.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=q.device)
+    if scale is None:
+        scale = d ** -0.5
+    rc = load().gqa_attention_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_lens), _ptr(sink), _ptr(out),
+                                          _ptr(lse), B, Hq, Hkv, Tq, Tkv, d, float(scale), int(bool(causal)),
+                                          _stream(stream))
+    _check("gqa_attention_fwd_noalloc", rc)
     return out, lse
 
 

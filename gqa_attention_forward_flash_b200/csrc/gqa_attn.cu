@@ -432,8 +432,126 @@ extern "C" const char* gqa_status_string(int status) {
         case GQA_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
         case GQA_ERR_UNSUPPORTED: return "unsupported head dim or GPU";
         case GQA_ERR_KVLEN: return "a kv_lens value was outside [0, Tkv] and was clamped";
+        case GQA_ERR_SCRATCH: return "the problem needs more scratch than the fixed allocation-free array holds";
         default: return "unknown status";
     }
 }
 
 extern "C" int gqa_version(void) { return 100; }
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of gqa_attention_fwd.
+//
+// gqa_attention_fwd grows a per-device scratch buffer with cudaMalloc the first
+// time it meets a problem that needs more room.  Some callers cannot allow that:
+// an engine that hands all device memory to its own pools at start-up and must
+// not see the driver allocate behind its back, a caller running inside a section
+// where an allocation (which may synchronise the device) is forbidden, or a host
+// integration that has no allocator at all.  For them this entry point keeps the
+// split-partial scratch in one fixed array compiled into this library, so every
+// GPU that loads the library holds it until the process exits.
+namespace gqa {
+namespace {
+
+constexpr size_t kNaCounterInts = 65536;                         // merge tickets: at most this many row-blocks
+constexpr size_t kNaErrOffset = kNaCounterInts * sizeof(int);    // device error word
+constexpr size_t kNaLseOffset = kNaErrOffset + 256;
+constexpr size_t kNaLseFloats = static_cast<size_t>(2) * kMaxCtas * 2 * BM;  // 2 slots x 256 rows per CTA
+constexpr size_t kNaPartOffset = kNaLseOffset + kNaLseFloats * sizeof(float);
+constexpr size_t kNaPartBytes = static_cast<size_t>(20) << 20;  // fp32 partial O: 20 MiB
+constexpr size_t kNaBytes = kNaPartOffset + kNaPartBytes;       // about 21.3 MiB in all
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNaBytes];
+
+struct NoAllocDevice {
+    bool ready = false;
+    unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+    int sm_count = 0;
+    int cc_major = 0;
+    long long clock_khz = 0;
+};
+NoAllocDevice g_na_dev[kMaxDevices];
+
+// Once per device, with that device current: the array's device address (the
+// host-side name g_noalloc_scratch is only a stand-in, not an address a kernel
+// may use), the SM count and clock, and the tensor-map encoder.
+int noalloc_setup(NoAllocDevice** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GQA_ERR_CUDA;
+    NoAllocDevice& s = g_na_dev[dev];
+    if (!s.ready) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return GQA_ERR_CUDA;
+        int sms = 0, major = 0, khz = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return GQA_ERR_CUDA;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return GQA_ERR_CUDA;
+        if (cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev) != cudaSuccess || khz <= 0) khz = 2000000;
+        if (!g_encode) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || fn == nullptr)
+                return GQA_ERR_CUDA;
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+        s.scratch = static_cast<unsigned char*>(ptr);
+        s.sm_count = sms;
+        s.cc_major = major;
+        s.clock_khz = khz;
+        s.ready = true;
+    }
+    *out = &s;
+    return GQA_OK;
+}
+
+}  // namespace
+}  // namespace gqa
+
+extern "C" int gqa_attention_fwd_noalloc(const void* q, const void* k, const void* v, const int32_t* kv_lens,
+                                         const float* sink, void* out, float* lse, int B, int Hq, int Hkv, int Tq,
+                                         int Tkv, int d, float scale, int causal, gqa_stream_t stream) {
+    int rc = check_common(q, k, v, B, Hq, Hkv, Tq, Tkv, d, scale);
+    if (rc) return rc;
+    if (B == 0 || Tq == 0) return GQA_OK;
+    if (!out) return GQA_ERR_NULL;
+    if (!aligned16(out) || (lse && !aligned16(lse))) return GQA_ERR_ALIGN;
+    if (d == 512) return GQA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    NoAllocDevice* s = nullptr;
+    rc = noalloc_setup(&s);
+    if (rc) return rc;
+    if (s->cc_major != 10) return GQA_ERR_UNSUPPORTED;
+    Params p;
+    long long ms = 1000;
+    if (const char* e = std::getenv("GQA_WAIT_TIMEOUT_MS")) {
+        const long long v2 = std::atoll(e);
+        if (v2 > 0) ms = v2;
+    }
+    fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale, causal, kv_lens, sink, out, lse, 0, s->clock_khz * ms);
+    choose_geometry(p);
+    if (p.W > static_cast<long long>(kNaCounterInts)) return GQA_ERR_SCRATCH;
+    // as many CTAs (one per SM) as the fixed partial area can give two slots each
+    const size_t rows_per_slot = static_cast<size_t>(BM) * p.RBQ;
+    const size_t per_cta = 2 * rows_per_slot * static_cast<size_t>(d) * sizeof(float);
+    long long NC = s->sm_count < kMaxCtas ? s->sm_count : kMaxCtas;
+    if (static_cast<long long>(kNaPartBytes / per_cta) < NC) NC = static_cast<long long>(kNaPartBytes / per_cta);
+    if (!kv_lens) {
+        long long tot = 0;
+        for (int qw = 0; qw < p.QW; ++qw) tot += qtile_ntiles(p, qw, Tkv);
+        tot *= p.U;
+        if (tot < NC) NC = tot;
+    }
+    if (NC < 1) return GQA_ERR_SCRATCH;
+    unsigned char* base = s->scratch;
+    p.mode = 0;
+    p.part_o = reinterpret_cast<float*>(base + kNaPartOffset);
+    p.part_lse = reinterpret_cast<float*>(base + kNaLseOffset);
+    p.counters = reinterpret_cast<int*>(base);
+    p.err = reinterpret_cast<int*>(base + kNaErrOffset);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // the array keeps the last call's contents: the merge tickets and the error
+    // word must start at zero
+    if (cudaMemsetAsync(base, 0, static_cast<size_t>(p.W) * sizeof(int), st) != cudaSuccess) return GQA_ERR_CUDA;
+    if (cudaMemsetAsync(base + kNaErrOffset, 0, sizeof(int), st) != cudaSuccess) return GQA_ERR_CUDA;
+    return dispatch_fwd(p, q, k, v, static_cast<int>(NC), st);
+}

@@ -74,7 +74,8 @@ typedef enum {
     GQA_ERR_CUDA = -5,        /* a CUDA runtime/driver call failed */
     GQA_ERR_TIMEOUT = -6,     /* a bounded wait inside a kernel ran out (device-reported) */
     GQA_ERR_UNSUPPORTED = -7, /* head dim not in {64,128,256,512}, or the GPU is not sm_100 */
-    GQA_ERR_KVLEN = -8        /* a kv_lens value was outside [0, Tkv] (device-reported, clamped) */
+    GQA_ERR_KVLEN = -8,       /* a kv_lens value was outside [0, Tkv] (device-reported, clamped) */
+    GQA_ERR_SCRATCH = -9      /* gqa_attention_fwd_noalloc: the problem exceeds its fixed scratch */
 } gqa_status;
 
 #define GQA_MAX_SPLITS 256
@@ -115,6 +116,35 @@ int gqa_attention_fwd_partial(const void *q, const void *k, const void *v, const
 int gqa_splitkv_combine(const float *o_part, const float *lse_part, int num_splits,
                         const float *sink, void *out, float *lse, int B, int Hq, int Tq, int d,
                         gqa_stream_t stream);
+
+/*
+ * gqa_attention_fwd without any device allocation.  The pages have no
+ * counterpart to this entry point; it exists for callers that cannot let a
+ * library allocate device memory: engines that carve all of HBM into their own
+ * pools at start-up, code running where an allocation (which may synchronise the
+ * device) is not allowed, and hosts without a device allocator.
+ *
+ * Same arguments, result and validation as gqa_attention_fwd.  The split
+ * partials that gqa_attention_fwd keeps in a cudaMalloc'd buffer live here in
+ * one fixed array inside the library (about 21.3 MiB: 20 MiB of fp32 partial
+ * rows, their lse values, 65536 merge tickets and an error word), held by every
+ * GPU that loads the library until the process exits.  Limits: at most 65536
+ * row-blocks (a row-block is 128 packed query rows of one KV head, 256 when a KV
+ * head has more than 128 packed rows), else GQA_ERR_SCRATCH; the grid uses at
+ * most as many CTAs as the array has two partial slots for, which for head
+ * dim 128 with more than 128 packed rows per KV head is fewer than the SM count.
+ * The first call on a device looks up the array's device address and the SM
+ * count (no allocation); make that first call outside any stream capture.
+ * Every call on a device shares the array and leaves its contents behind: each
+ * call clears, on its stream, the tickets and the error word it uses, and calls
+ * whose executions overlap on the GPU (on streams the caller does not order)
+ * race on it.  Device-side errors (an expired bounded
+ * wait, a clamped kv_lens value) are recorded in the array's error word and not
+ * reported; diagnose with gqa_attention_fwd and gqa_get_device_error.
+ */
+int gqa_attention_fwd_noalloc(const void *q, const void *k, const void *v, const int32_t *kv_lens,
+                              const float *sink, void *out, float *lse, int B, int Hq, int Hkv,
+                              int Tq, int Tkv, int d, float scale, int causal, gqa_stream_t stream);
 
 /*
  * Waits for `stream`, then returns (and clears) the first error a kernel of
