@@ -147,10 +147,18 @@ using C2_64_DQ = Fwd2Cfg<64, 4, 4, 2>;
 using C2_128_SK = Fwd2Cfg<128, 3, 3, 1>;
 using C2_128_DQ = Fwd2Cfg<128, 3, 2, 2>;
 using Cfg256 = FwdCfg<256, 64, 3, 2, 1>;
+// Head dim 512: O (128 x 512 fp32) fills a whole TMEM, so O's columns are split
+// over a pair of CTAs (DSPLIT = 2) that each compute the full S.
+using Cfg512 = FwdCfg<512, 32, 2, 2, 1, 2>;
+
+int dsplit_for(int d) { return d == 512 ? Cfg512::DSPLIT : 1; }
 
 // Tile geometry of the kernel that will serve these sizes.
 void choose_geometry(Params& p) {
-    if (p.d == 256) {
+    if (p.d == 512) {
+        p.BN = Cfg512::BN;
+        p.RBQ = 1;
+    } else if (p.d == 256) {
         p.BN = Cfg256::BN;
         p.RBQ = 1;
     } else {
@@ -215,6 +223,7 @@ int dispatch_fwd(const Params& p, const void* q, const void* k, const void* v, i
             return p.RBQ == 1 ? launch_fwd<C2_128_SK, true>(p, q, k, v, grid, stream, e0, e1)
                               : launch_fwd<C2_128_DQ, true>(p, q, k, v, grid, stream, e0, e1);
         case 256: return launch_fwd<Cfg256, false>(p, q, k, v, grid, stream, e0, e1);
+        case 512: return launch_fwd<Cfg512, false>(p, q, k, v, grid, stream, e0, e1);
         default: return GQA_ERR_UNSUPPORTED;
     }
 }
@@ -271,7 +280,6 @@ extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, co
     if (B == 0 || Tq == 0) return GQA_OK;
     if (!out) return GQA_ERR_NULL;
     if (!aligned16(out) || (lse && !aligned16(lse))) return GQA_ERR_ALIGN;
-    if (d == 512) return GQA_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lk(g_mu);
     DeviceState* s = nullptr;
     rc = get_state(&s);
@@ -280,8 +288,10 @@ extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, co
     Params p;
     fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale, causal, kv_lens, sink, out, lse, 0, timeout_cycles(*s));
     choose_geometry(p);
-    // grid: one CTA per SM; with host-known lengths never more CTAs than tiles
-    int NC = s->sm_count < kMaxCtas ? s->sm_count : kMaxCtas;
+    // grid: one CTA per SM (NC groups of DSPLIT CTAs); with host-known lengths never
+    // more groups than tiles
+    const int ds = dsplit_for(d);
+    int NC = (s->sm_count < kMaxCtas ? s->sm_count : kMaxCtas) / ds;
     if (!kv_lens) {
         long long tot = 0;
         for (int qw = 0; qw < p.QW; ++qw) tot += qtile_ntiles(p, qw, Tkv);
@@ -289,12 +299,12 @@ extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, co
         if (tot < NC) NC = static_cast<int>(tot);
     }
     if (NC < 1) NC = 1;
-    const size_t slot_rows = static_cast<size_t>(2 * NC) * BM * p.RBQ;
-    const size_t slot_o = slot_rows * d * sizeof(float);
+    const size_t slot_rows = static_cast<size_t>(2 * NC) * ds * BM * p.RBQ;
+    const size_t slot_o = slot_rows * (d / ds) * sizeof(float);
     const size_t slot_l = slot_rows * sizeof(float);
     rc = ensure_scratch(*s, slot_o + slot_l);
     if (rc) return rc;
-    rc = ensure_counters(*s, p.W);
+    rc = ensure_counters(*s, p.W * ds);
     if (rc) return rc;
     char* base = static_cast<char*>(s->scratch);
     p.mode = 0;
@@ -309,7 +319,7 @@ extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, co
         cudaGetDevice(&dev);
         if (dev == g_prof.dev) ev = g_prof.ev[g_prof.n++];
     }
-    rc = dispatch_fwd(p, q, k, v, NC, st, ev ? ev[0] : nullptr, ev ? ev[1] : nullptr);
+    rc = dispatch_fwd(p, q, k, v, NC * ds, st, ev ? ev[0] : nullptr, ev ? ev[1] : nullptr);
     if (rc) return rc;
     if (ev && cudaEventRecord(ev[2], st) != cudaSuccess) return GQA_ERR_CUDA;
     return GQA_OK;
@@ -324,7 +334,6 @@ extern "C" int gqa_attention_fwd_partial(const void* q, const void* k, const voi
     if (B == 0 || Tq == 0) return GQA_OK;
     if (!o_part || !lse_part) return GQA_ERR_NULL;
     if (!aligned16(o_part) || !aligned16(lse_part)) return GQA_ERR_ALIGN;
-    if (d == 512) return GQA_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lk(g_mu);
     DeviceState* s = nullptr;
     rc = get_state(&s);
@@ -334,7 +343,7 @@ extern "C" int gqa_attention_fwd_partial(const void* q, const void* k, const voi
     fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale, causal, kv_lens, nullptr, nullptr, nullptr, 0,
                 timeout_cycles(*s));
     choose_geometry(p);
-    const long long grid = p.W * num_splits;
+    const long long grid = p.W * num_splits * dsplit_for(d);
     if (grid >= (1ll << 31)) return GQA_ERR_SHAPE;
     p.mode = 1;
     p.num_splits = num_splits;

@@ -295,20 +295,28 @@ struct SegWalker {
 
 // ------------------------------------------------------------------ kernel config
 
-template <int D_, int BN_, int STK_, int STV_, int QBUF_>
+// DSPLIT > 1 splits O's columns over DSPLIT CTAs that walk the same key tiles:
+// each computes the full S = Q K^T (all D columns of Q and K) but accumulates
+// only its DO = D / DSPLIT columns of O, so a 128 x 512 fp32 O never has to fit
+// one SM's 512 TMEM columns.
+template <int D_, int BN_, int STK_, int STV_, int QBUF_, int DSPLIT_ = 1>
 struct FwdCfg {
-    static constexpr int D = D_, BN = BN_, STK = STK_, STV = STV_, QBUF = QBUF_;
-    static_assert(D % 64 == 0 && D <= 256, "head dim");
-    static_assert(BN == 64 || BN == 128, "key tile");
-    static constexpr int NBOX = D / 64;                 // 64-column swizzle boxes per row
+    static constexpr int D = D_, BN = BN_, STK = STK_, STV = STV_, QBUF = QBUF_, DSPLIT = DSPLIT_;
+    static constexpr int DO = D / DSPLIT;               // O columns owned by one CTA
+    static_assert(D % 64 == 0 && D <= 512 && DO <= 256 && DO % 64 == 0, "head dim");
+    static_assert(BN == 32 || BN == 64 || BN == 128, "key tile");
+    static constexpr int HALVES = (BN >= 64) ? 2 : 1;   // softmax column groups per row
+    static constexpr int NBOX = D / 64;                 // 64-column swizzle boxes per Q/K row
+    static constexpr int VBOX = DO / 64;                // boxes of the V columns this CTA reads
     static constexpr int Q_BOX = BM * 128;              // bytes of one Q box
     static constexpr int Q_BYTES = NBOX * Q_BOX;
     static constexpr int KV_BOX = BN * 128;
-    static constexpr int KV_BYTES = NBOX * KV_BOX;      // one K (or V) tile
+    static constexpr int KV_BYTES = NBOX * KV_BOX;      // one K tile
+    static constexpr int V_BYTES = VBOX * KV_BOX;       // one V tile (this CTA's columns)
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + QBUF * Q_BYTES;
     static constexpr int OFF_V = OFF_K + STK * KV_BYTES;
-    static constexpr int OFF_BAR = OFF_V + STV * KV_BYTES;
+    static constexpr int OFF_BAR = OFF_V + STV * V_BYTES;
     // barrier indices
     static constexpr int B_QFULL = 0;
     static constexpr int B_QEMPTY = B_QFULL + QBUF;
@@ -328,14 +336,14 @@ struct FwdCfg {
     static constexpr int SMEM_USED = OFF_MISC + MISC_BYTES;
     static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack to align the base to 1024
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-    // TMEM columns: O [0, D), S[2] of BN fp32 columns, P[2] of BN/2 columns (bf16 pairs)
+    // TMEM columns: O [0, DO), S[2] of BN fp32 columns, P[2] of BN/2 columns (bf16 pairs)
     static constexpr uint32_t TM_O = 0;
-    static constexpr uint32_t TM_S = D;
-    static constexpr uint32_t TM_P = D + 2 * BN;
+    static constexpr uint32_t TM_S = DO;
+    static constexpr uint32_t TM_P = DO + 2 * BN;
     static constexpr uint32_t TM_COLS = 512;
-    static_assert(D + 3 * BN <= 512, "TMEM budget");
+    static_assert(DO + 3 * BN <= 512, "TMEM budget");
     static constexpr uint32_t IDESC_S = ptx::umma_idesc_bf16_f32(BM, BN, false, false);
-    static constexpr uint32_t IDESC_PV = ptx::umma_idesc_bf16_f32(BM, D, false, true);
+    static constexpr uint32_t IDESC_PV = ptx::umma_idesc_bf16_f32(BM, DO, false, true);
 };
 
 struct Misc {
@@ -418,8 +426,10 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int cta = blockIdx.x;
-    const int NC = gridDim.x;
+    // CTAs come in groups of DSPLIT that walk the same work; ho picks the O columns
+    const int ho = static_cast<int>(blockIdx.x) % C::DSPLIT;
+    const int cta = static_cast<int>(blockIdx.x) / C::DSPLIT;
+    const int NC = static_cast<int>(gridDim.x) / C::DSPLIT;
 
     // ---------------------------------------------------------------- setup
     if (threadIdx.x == 0) {
@@ -528,11 +538,11 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     ok = wait_bar(bar(C::B_VEMPTY + st), ((g / C::STV) & 1) ^ 1, misc, p);
                     if (!ok) break;
                     const int y = static_cast<int>(rb.kv_row0 + static_cast<long long>(t) * C::BN);
-                    ptx::mbar_arrive_expect_tx(bar(C::B_VFULL + st), C::NBOX * p.kv_box_rows * 128);
+                    ptx::mbar_arrive_expect_tx(bar(C::B_VFULL + st), C::VBOX * p.kv_box_rows * 128);
                     ++v_issued[st];
-                    for (int bx = 0; bx < C::NBOX; ++bx)
-                        ptx::tma_load_2d(sbase + C::OFF_V + st * C::KV_BYTES + bx * C::KV_BOX, &tm_v, bx * 64, y,
-                                         bar(C::B_VFULL + st), pol_kv);
+                    for (int bx = 0; bx < C::VBOX; ++bx)
+                        ptx::tma_load_2d(sbase + C::OFF_V + st * C::V_BYTES + bx * C::KV_BOX, &tm_v,
+                                         ho * C::DO + bx * 64, y, bar(C::B_VFULL + st), pol_kv);
                 }
             }
             for (int i = 0; i < C::STV; ++i) drain_bar(bar(C::B_VFULL + i), v_issued[i], p.timeout_cycles);
@@ -557,7 +567,7 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const int st = gp % C::STV;
                 if (!wait_bar(bar(C::B_VFULL + st), (gp / C::STV) & 1, misc, p)) return false;
                 ptx::tc_fence_after();
-                const uint32_t vbase = sbase + C::OFF_V + st * C::KV_BYTES;
+                const uint32_t vbase = sbase + C::OFF_V + st * C::V_BYTES;
                 const uint32_t tm_p = tmem + C::TM_P + pb * (C::BN / 2);
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk) {
@@ -618,8 +628,8 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int half = (warp - 2) >> 2;      // which half of the key columns / O columns
         const int lrow = quad * 32 + lane;     // TMEM lane = row of the MMA tile
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-        constexpr int HB = C::BN / 2;          // key columns per half
-        constexpr int HD = C::D / 2;           // O columns per half
+        constexpr int HB = C::BN / C::HALVES;  // key columns per half
+        constexpr int HD = C::DO / C::HALVES;  // O columns per half
         const uint32_t tm_o = tmem + lane_off + C::TM_O + half * HD;
         const int stid = threadIdx.x - 64;     // 0..255 among the softmax threads
         // Barrier over the 256 softmax threads on an mbarrier with a bounded wait, so
@@ -652,6 +662,8 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 valid = lrow < rb.rows_valid;
                 active = quad * 32 < rb.rows_valid;
             }
+            // with a single column group the second group's warps only keep the barrier counts
+            active = active && half < C::HALVES;
             const int rp = rb.qt * BM + rloc;   // packed row inside the unit
             const int hl = valid ? rp / p.Tq : 0;
             const int i = valid ? rp % p.Tq : 0;
@@ -701,7 +713,7 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     // other half: only its maximum is needed
                     const int olim = lim_all - (half ^ 1) * HB;
 #pragma unroll
-                    for (int c = 0; c < HB / 32; ++c) {
+                    for (int c = 0; c < (C::HALVES == 2 ? HB / 32 : 0); ++c) {
                         uint32_t r[32];
                         ptx::tmem_ld32(tm_s + (half ^ 1) * HB + c * 32, r);
                         ptx::tmem_wait_ld();
@@ -785,11 +797,11 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     if (!ok) break;
                     int z0 = sg.n - t * C::BN;
                     z0 = z0 < 0 ? 0 : z0;
-                    uint8_t* vt = smem + C::OFF_V + st * C::KV_BYTES;
-                    const int chunks = (C::BN - z0) * C::NBOX * 8;  // 16-byte chunks
+                    uint8_t* vt = smem + C::OFF_V + st * C::V_BYTES;
+                    const int chunks = (C::BN - z0) * C::VBOX * 8;  // 16-byte chunks
                     for (int q = stid; q < chunks; q += NSOFT) {
-                        const int r = z0 + q / (C::NBOX * 8);
-                        const int rem = q % (C::NBOX * 8);
+                        const int r = z0 + q / (C::VBOX * 8);
+                        const int rem = q % (C::VBOX * 8);
                         *reinterpret_cast<uint4*>(vt + (rem >> 3) * C::KV_BOX + r * 128 + (rem & 7) * 16) =
                             make_uint4(0, 0, 0, 0);
                     }
@@ -831,7 +843,7 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             const long long fr = rb.q_row0 + rloc;  // flat row (b*Hq + h)*Tq + i when valid
             if (sg.kind == 0) {
-                __nv_bfloat16* dst = p.out + fr * C::D + half * HD;
+                __nv_bfloat16* dst = p.out + fr * C::D + ho * C::DO + half * HD;
                 if (active) {
 #pragma unroll 1
                     for (int c = 0; c < HD / 32; ++c) {
@@ -851,15 +863,17 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         }
                     }
                 }
-                if (valid && half == 0 && p.lse != nullptr) p.lse[fr] = lse_v;
+                if (valid && half == 0 && ho == 0 && p.lse != nullptr) p.lse[fr] = lse_v;
             } else {
+                // stream-K slots hold [BM rows][DO columns] per CTA of a DSPLIT group
                 float* dst;
                 float* dl;
                 if (sg.kind == 1) {
-                    dst = p.part_o + (static_cast<long long>(sg.slot) * BM + rloc) * C::D + half * HD;
-                    dl = p.part_lse + static_cast<long long>(sg.slot) * BM + rloc;
+                    const long long slot = static_cast<long long>(sg.slot) * C::DSPLIT + ho;
+                    dst = p.part_o + (slot * BM + rloc) * C::DO + half * HD;
+                    dl = p.part_lse + slot * BM + rloc;
                 } else {
-                    dst = p.part_o + (fr * p.num_splits + sg.slot) * C::D + half * HD;
+                    dst = p.part_o + (fr * p.num_splits + sg.slot) * C::D + ho * C::DO + half * HD;
                     dl = p.part_lse + fr * p.num_splits + sg.slot;
                 }
                 if (active) {
@@ -885,7 +899,7 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         }
                     }
                 }
-                if (valid && half == 0) __stcg(dl, lse_v);
+                if (valid && half == 0 && (sg.kind == 1 || ho == 0)) __stcg(dl, lse_v);
 
                 if (sg.kind == 1) {
                     __threadfence();  // this thread's partial rows are visible before the ticket
@@ -899,7 +913,7 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         for (int cc = c_first; cc <= c_last; ++cc)
                             ncontrib += span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC);
                         __threadfence();
-                        const int old = atomicAdd(p.counters + sg.w, 1);
+                        const int old = atomicAdd(p.counters + static_cast<long long>(sg.w) * C::DSPLIT + ho, 1);
                         const int last = (old == ncontrib - 1);
                         if (last) __threadfence();
                         misc->merge_flag = last;
@@ -914,23 +928,25 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             float L = (p.sink != nullptr) ? __ldg(p.sink + hr) : -INFINITY;
                             for (int cc = c_first; cc <= c_last; ++cc) {
                                 if (!(span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC))) continue;
-                                L = fmaxf(L, __ldcg(p.part_lse + merge_slot(cc, c_first, c0_first) * BM + r));
+                                const long long sl = merge_slot(cc, c_first, c0_first) * C::DSPLIT + ho;
+                                L = fmaxf(L, __ldcg(p.part_lse + sl * BM + r));
                             }
                             float lt = -INFINITY;
                             if (L != -INFINITY) {
                                 float z = (p.sink != nullptr) ? __expf(__ldg(p.sink + hr) - L) : 0.f;
                                 for (int cc = c_first; cc <= c_last; ++cc) {
                                     if (!(span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC))) continue;
-                                    z += __expf(__ldcg(p.part_lse + merge_slot(cc, c_first, c0_first) * BM + r) - L);
+                                    const long long sl = merge_slot(cc, c_first, c0_first) * C::DSPLIT + ho;
+                                    z += __expf(__ldcg(p.part_lse + sl * BM + r) - L);
                                 }
                                 lt = L + __logf(z);
                             }
                             misc->mlse[r] = lt;
-                            if (p.lse != nullptr) p.lse[rb.q_row0 + r] = lt;
+                            if (p.lse != nullptr && ho == 0) p.lse[rb.q_row0 + r] = lt;
                         }
                         if (!xsync()) { ok = false; break; }
                         // weighted sum of the partials, 8 columns per item
-                        constexpr int C8 = C::D / 8;
+                        constexpr int C8 = C::DO / 8;
                         for (int it = stid; it < rb.rows_valid * C8; it += NSOFT) {
                             const int r = it / C8, c8 = it % C8;
                             const float lt = misc->mlse[r];
@@ -938,20 +954,20 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             if (lt != -INFINITY) {
                                 for (int cc = c_first; cc <= c_last; ++cc) {
                                     if (!(span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC))) continue;
-                                    const long long sl = merge_slot(cc, c_first, c0_first);
+                                    const long long sl = merge_slot(cc, c_first, c0_first) * C::DSPLIT + ho;
                                     const float wgt = __expf(__ldcg(p.part_lse + sl * BM + r) - lt);
                                     const float4* src =
-                                        reinterpret_cast<const float4*>(p.part_o + (sl * BM + r) * C::D + 8 * c8);
+                                        reinterpret_cast<const float4*>(p.part_o + (sl * BM + r) * C::DO + 8 * c8);
                                     const float4 a = __ldcg(src), b = __ldcg(src + 1);
                                     acc[0] += wgt * a.x; acc[1] += wgt * a.y; acc[2] += wgt * a.z; acc[3] += wgt * a.w;
                                     acc[4] += wgt * b.x; acc[5] += wgt * b.y; acc[6] += wgt * b.z; acc[7] += wgt * b.w;
                                 }
                             }
-                            *reinterpret_cast<uint4*>(p.out + (rb.q_row0 + r) * C::D + 8 * c8) =
+                            *reinterpret_cast<uint4*>(p.out + (rb.q_row0 + r) * C::D + ho * C::DO + 8 * c8) =
                                 make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
                                            pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
                         }
-                        if (stid == 0) p.counters[sg.w] = 0;  // ready for the next call
+                        if (stid == 0) p.counters[static_cast<long long>(sg.w) * C::DSPLIT + ho] = 0;  // ready for the next call
                     }
                 }
             }

@@ -35,6 +35,8 @@ SMALL = {
     "tq_gt_len_empty_rows": Workload("empty", B=2, Hq=4, Hkv=2, Tq=40, Tkv=64, d=128, causal=True,
                                      kv_len=20, nan_pad=True, sink=True, seed=11),
     "noncausal_prefill_d128": Workload("nc", B=1, Hq=8, Hkv=1, Tq=130, Tkv=515, d=128, seed=12),
+    "d512_sink_nan": shrink(W["wide_head_sink_decode"], B=2, Tkv=700, kv_len=631),
+    "d512_mha_noncausal": Workload("d512", B=1, Hq=2, Hkv=2, Tq=70, Tkv=200, d=512, seed=20),
 }
 
 
@@ -127,9 +129,9 @@ def test_deterministic_bitwise():
     assert binding.gqa_get_device_error() == 0
 
 
-@pytest.mark.parametrize("splits", [1, 3, 8])
-def test_forced_splits_then_combine(splits):
-    w = Workload("split", B=2, Hq=8, Hkv=2, Tq=3, Tkv=900, d=128, causal=True, sink=True, ragged=True,
+@pytest.mark.parametrize("splits,d", [(1, 128), (3, 128), (8, 128), (3, 512), (2, 64), (2, 256)])
+def test_forced_splits_then_combine(splits, d):
+    w = Workload("split", B=2, Hq=8, Hkv=2, Tq=3, Tkv=900, d=d, causal=True, sink=True, ragged=True,
                  nan_pad=True, seed=16)
     inp = make_inputs(w)
     t = to_device(inp)
@@ -161,7 +163,7 @@ def test_combine_kernel_on_oracle_partials():
 
 # ------------------------------------------------------------------ full size, sampled rows
 
-FULL = ["batched_decode", "short_q_long_kv", "full_causal_prefill"]
+FULL = ["batched_decode", "short_q_long_kv", "full_causal_prefill", "wide_head_sink_decode"]
 
 
 @pytest.mark.parametrize("name", FULL)
