@@ -322,7 +322,7 @@ def run_ours(args, w, ws, rank, local):
     torch.cuda.synchronize(dev)
     barrier(ws)
     clocks = sampler.stop()
-    main_ms, comb_ms = binding.gqa_profile_take()
+    main_ms = binding.gqa_profile_take()
     err = binding.gqa_get_device_error(stream)
     if err != 0:
         raise RuntimeError("device error %d in the timed steps" % err)
@@ -342,8 +342,7 @@ def run_ours(args, w, ws, rank, local):
     traffic = traffic_for(w)
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": traffic, "peak_source": peak_src + (" (burst)" if bound == "tensor" else ""),
-                "kernel": "gqa_fwd_kernel", "kernel_ms": main_avg,
-                "combine_ms": statistics.mean(comb_ms) if comb_ms else None,
+                "kernel": main_kernel_name(w), "kernel_ms": main_avg, "launches_per_step": 1,
                 "algorithmic_bytes": nbytes, "algorithmic_flops": nflops}
 
     # end to end through the public API with host buffers
@@ -361,7 +360,7 @@ def run_ours(args, w, ws, rank, local):
             "metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(w),
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": len(main_ms),
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -412,18 +411,40 @@ def run_e2e(args, w, inp, dev, stream, nbytes, nflops, ws):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
 
 
+def main_kernel_name(w: Workload) -> str:
+    """The kernel gqa_attention_fwd launches for this head dim (its only launch)."""
+    return "gqa_fwd2_kernel" if w.d <= 128 else "gqa_fwd_kernel"
+
+
+def kernel_source_digest() -> str:
+    """sha256 over the library's CUDA sources (file name + contents, sorted)."""
+    import hashlib
+    h = hashlib.sha256()
+    cs = os.path.join(ROOT, "gqa_attention_forward_flash_b200", "csrc")
+    for name in sorted(os.listdir(cs)):
+        if name.endswith((".cu", ".cuh")):
+            h.update(name.encode())
+            with open(os.path.join(cs, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()
+
+
 def traffic_for(w: Workload):
-    """DRAM bytes per launch of the main kernel from a committed ncu summary of
-    this exact kernel build and workload, if present (profiles/traffic.json)."""
+    """DRAM bytes (read + write) per launch of the main kernel, from the ncu
+    capture recorded in profiles/traffic.json, or None when there is none for
+    this workload or the kernel sources changed since it was taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     try:
         with open(p) as f:
             d = json.load(f)
-        return d.get(w.name)
     except (OSError, ValueError):
         return None
+    if d.get("source_sha256") != kernel_source_digest():
+        return None
+    e = d.get("workloads", {}).get(w.name)
+    return None if e is None else e.get("bytes_per_launch")
 
 
 def main():

@@ -31,7 +31,7 @@ SIGNATURES = {
     "gqa_splitkv_combine": (_I, [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
     "gqa_get_device_error": (_I, [_P]),
     "gqa_profile_begin": (_I, []),
-    "gqa_profile_take": (_I, [_P, _P, _I, _P]),
+    "gqa_profile_take": (_I, [_P, _I, _P]),
     "gqa_status_string": (ctypes.c_char_p, [_I]),
     "gqa_version": (_I, []),
 }
@@ -167,12 +167,11 @@ def gqa_profile_begin() -> None:
 
 
 def gqa_profile_take(max_calls: int = 4096):
-    """Per-call (main kernel ms, combine kernel ms) since gqa_profile_begin."""
-    main = (ctypes.c_float * max_calls)()
-    comb = (ctypes.c_float * max_calls)()
+    """Per-call kernel durations (ms) since gqa_profile_begin."""
+    ms = (ctypes.c_float * max_calls)()
     n = ctypes.c_int(0)
-    _check("gqa_profile_take", load().gqa_profile_take(main, comb, max_calls, ctypes.byref(n)))
-    return list(main[:n.value]), list(comb[:n.value])
+    _check("gqa_profile_take", load().gqa_profile_take(ms, max_calls, ctypes.byref(n)))
+    return list(ms[:n.value])
 
 
 def gqa_status_string(status: int) -> str:

@@ -40,14 +40,14 @@ std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 
 // Optional per-launch timing (gqa_profile_*): events recorded on the launch
-// stream around the main kernel and around the combine kernel of each
+// stream right before and right after the one kernel of each
 // gqa_attention_fwd call, read back by gqa_profile_take.
 constexpr int kProfCap = 4096;
 struct Prof {
     bool on = false;
     int dev = -1;
     int n = 0;
-    cudaEvent_t ev[kProfCap][3];
+    cudaEvent_t ev[kProfCap][2];
     bool created = false;
 };
 Prof g_prof;
@@ -321,7 +321,6 @@ extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, co
     }
     rc = dispatch_fwd(p, q, k, v, NC * ds, st, ev ? ev[0] : nullptr, ev ? ev[1] : nullptr);
     if (rc) return rc;
-    if (ev && cudaEventRecord(ev[2], st) != cudaSuccess) return GQA_ERR_CUDA;
     return GQA_OK;
 }
 
@@ -395,18 +394,16 @@ extern "C" int gqa_profile_begin(void) {
     return GQA_OK;
 }
 
-extern "C" int gqa_profile_take(float* main_ms, float* combine_ms, int max_calls, int* n_calls) {
+extern "C" int gqa_profile_take(float* kernel_ms, int max_calls, int* n_calls) {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!n_calls) return GQA_ERR_NULL;
     g_prof.on = false;
     const int n = g_prof.n < max_calls ? g_prof.n : max_calls;
     for (int i = 0; i < n; ++i) {
-        if (cudaEventSynchronize(g_prof.ev[i][2]) != cudaSuccess) return GQA_ERR_CUDA;
-        float a = 0.f, b = 0.f;
+        if (cudaEventSynchronize(g_prof.ev[i][1]) != cudaSuccess) return GQA_ERR_CUDA;
+        float a = 0.f;
         if (cudaEventElapsedTime(&a, g_prof.ev[i][0], g_prof.ev[i][1]) != cudaSuccess) return GQA_ERR_CUDA;
-        if (cudaEventElapsedTime(&b, g_prof.ev[i][1], g_prof.ev[i][2]) != cudaSuccess) return GQA_ERR_CUDA;
-        if (main_ms) main_ms[i] = a;
-        if (combine_ms) combine_ms[i] = b;
+        if (kernel_ms) kernel_ms[i] = a;
     }
     *n_calls = n;
     g_prof.n = 0;

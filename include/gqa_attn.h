@@ -157,13 +157,14 @@ int gqa_get_device_error(gqa_stream_t stream);
 /*
  * Measurement hook (no counterpart on the pages; it only observes).  After
  * gqa_profile_begin, each gqa_attention_fwd call on the current device (up to
- * 4096 calls) records CUDA events on its own stream before and after its main
- * kernel and after its combine kernel.  gqa_profile_take stops recording, waits
- * for those events and writes, per call, the main kernel's and the combine
- * kernel's durations in ms (either array may be NULL) and the number of calls.
+ * 4096 calls) records CUDA events on its own stream right before and right
+ * after its kernel (one launch per call: the split-KV merge runs inside it).
+ * gqa_profile_take stops recording, waits for those events and writes, per
+ * call, the kernel's duration in ms into kernel_ms[0 .. *n_calls) (kernel_ms
+ * may be NULL; at most max_calls entries).
  */
 int gqa_profile_begin(void);
-int gqa_profile_take(float *main_ms, float *combine_ms, int max_calls, int *n_calls);
+int gqa_profile_take(float *kernel_ms, int max_calls, int *n_calls);
 
 /* A static English description of a status code. */
 const char *gqa_status_string(int status);
