@@ -23,8 +23,10 @@
 // lane's previous P from it; the tensor core executes one thread's MMAs in issue
 // order, which orders the overwrite after the read.
 //
-// Warps 0-3: lane 0 softmax; 4-7: lane 1 softmax; 8: TMA producers (lane 0: Q
-// and K ring, lane 16: V ring); 9: TMEM owner + MMA issuer; 10-11: idle.
+// Warps 0-3: lane 0 softmax; 4-7: lane 1 softmax; 8: Q and K producer (one
+// thread); 9: TMEM owner + MMA issuer; 10: split-segment ticket taker; 11: V
+// producer.  Each single-thread role has a warp of its own, so no role's spin
+// on a barrier delays another's issue.
 // Work split, logical-length masking, the sink, split partials and the
 // last-arriver merge follow the single-lane kernel (gqa_fwd_kernel.cuh).
 #pragma once
@@ -34,6 +36,7 @@ namespace gqa {
 
 constexpr int NUM_THREADS2 = 384;  // 12 warps = 3 warpgroups
 constexpr int NSOFT2 = 256;        // softmax threads (two warpgroups)
+constexpr int kMaxMergeSlots = 64; // pieces a row-block's merge lists in shared memory
 
 template <int D_, int STK_, int STV_, int RBQ_>
 struct Fwd2Cfg {
@@ -60,9 +63,11 @@ struct Fwd2Cfg {
     static constexpr int B_ODONE = B_PFULL + 2;     // [2 lanes]
     static constexpr int B_FINAL = B_ODONE + 2;
     static constexpr int B_XSYNC = B_FINAL + 1;
-    static constexpr int NBAR = B_XSYNC + 1;
+    static constexpr int B_MJOB = B_XSYNC + 1;   // [2] partial rows of split segment j written
+    static constexpr int B_MTICK = B_MJOB + 2;   // [2] ticket of split segment j taken
+    static constexpr int NBAR = B_MTICK + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr int MISC_BYTES = 2112;
+    static constexpr int MISC_BYTES = 2496;
     // the dynamic shared-memory window is required (and checked) to start 1024-aligned
     static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -85,6 +90,10 @@ struct Misc2 {
         float mlse[2 * BM];   // merged lse per packed row (in-kernel merge, later)
     };
     float st_l[2][BM];        // per-lane row sum
+    int nmerge;               // pieces of the row-block being merged
+    int mslot[kMaxMergeSlots];  // their partial slots
+    Seg jobs[2];              // this CTA's split segments (its first and last at most)
+    int ticket[2];            // 1: this CTA wrote the row-block's last piece and merges it
 };
 
 template <class C>
@@ -127,6 +136,10 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         ptx::mbar_init(bar(C::B_FINAL), 1);
         ptx::mbar_init(bar(C::B_XSYNC), NSOFT2 / 32);
+        for (int j = 0; j < 2; ++j) {
+            ptx::mbar_init(bar(C::B_MJOB + j), 1);
+            ptx::mbar_init(bar(C::B_MTICK + j), 1);
+        }
         misc->abort = 0;
         misc->merge_flag = 0;
         if (p.mode != 0) {
@@ -194,7 +207,7 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             for (int i = 0; i < C::STK; ++i) drain_bar(bar(C::B_KFULL + i), k_issued[i], p.timeout_cycles);
             drain_bar(bar(C::B_QFULL), q_issued, p.timeout_cycles);
-        } else if (warp == 8 && lane == 16) {
+        } else if (warp == 11 && lane == 0) {
             const uint64_t pol_kv = (p.QW == 1) ? ptx::policy_evict_first() : ptx::policy_evict_normal();
             SegWalker wk;
             wk.init(p, misc->span, cta);
@@ -268,6 +281,21 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
             while (ok && wk.next(p, sg)) {
                 if (sg.t1 <= sg.t0) continue;
+                // the previous segment's last PV goes out before this segment's Q is
+                // awaited: that segment's epilogue waits for the PV, and the new Q
+                // may still be in flight
+                if (C::RBQ == 1 && have_prev) {
+                    ok = issue_pv(prev_lane, prev_stv, prev_first, true, g - 1);
+                    if (!ok) break;
+                    ptx::umma_commit(bar(C::B_VEMPTY + prev_stv));
+                    have_prev = false;
+                }
+                if (C::RBQ == 2 && have_b) {
+                    ok = issue_pv(1, b_stv, b_first, false, 0);
+                    if (!ok) break;
+                    ptx::umma_commit(bar(C::B_VEMPTY + b_stv));
+                    have_b = false;
+                }
                 ok = wait_bar(bar(C::B_QFULL), seg_i & 1, wmisc, p);
                 if (!ok) break;
                 const uint32_t qbase = sbase + C::OFF_Q;
@@ -324,6 +352,31 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             ptx::umma_commit(bar(C::B_FINAL));
             drain_bar(bar(C::B_FINAL), 1, p.timeout_cycles);
         }
+        // ------------------------------------------------------------ ticket taker
+        // For each split segment: once the softmax warps have written its partial
+        // rows, publish them (release fence) and count this CTA's piece of the
+        // row-block; the CTA whose count completes it merges the pieces.  The
+        // softmax warps do not wait for this until their last segment is done.
+        else if (warp == 10 && lane == 0) {
+            SegWalker wk;
+            wk.init(p, misc->span, cta);
+            Seg sg;
+            int j = 0;
+            const long long tot = misc->span.tot;
+            while (j < 2 && wk.next(p, sg)) {
+                if (sg.kind != 1) continue;
+                if (!wait_bar(bar(C::B_MJOB + j), 0, wmisc, p)) break;
+                const int c_first = cta_of(sg.pw, tot, NC);
+                const int c_last = cta_of(sg.pw + sg.ntiles - 1, tot, NC);
+                int ncontrib = 0;
+                for (int cc = c_first; cc <= c_last; ++cc) ncontrib += span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC);
+                __threadfence();
+                const int old = atomicAdd(p.counters + sg.w, 1);
+                misc->ticket[j] = (old == ncontrib - 1);
+                ptx::mbar_arrive(bar(C::B_MTICK + j));
+                ++j;
+            }
+        }
     }
     // ---------------------------------------------------------------- softmax lanes
     else {
@@ -350,6 +403,7 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         uint32_t g = 0;
         uint32_t cnt = 0;  // tiles this lane has processed (barrier phases)
         bool ok = true;
+        int njob = 0;      // split segments handed to the ticket taker
 
         while (ok && wk.next(p, sg)) {
             const RB rb = rb_of(p, sg.w);
@@ -583,29 +637,113 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
             // both lanes' O reads are done before the next segment's first PVs
-            // overwrite them; the partial rows are complete before the ticket
-            if (sg.kind == 1) __threadfence();
+            // overwrite them; a split segment's partial rows are written
             if (!xsync()) { ok = false; break; }
-
-            if (sg.kind == 1) {
-                const long long tot = misc->span.tot;
-                const int c_first = cta_of(sg.pw, tot, NC);
-                const int c_last = cta_of(sg.pw + sg.ntiles - 1, tot, NC);
+            if (sg.kind == 1 && njob < 2) {
                 if (stid == 0) {
-                    int ncontrib = 0;
-                    for (int cc = c_first; cc <= c_last; ++cc)
-                        ncontrib += span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC);
-                    __threadfence();
-                    const int old = atomicAdd(p.counters + sg.w, 1);
-                    const int last = (old == ncontrib - 1);
-                    if (last) __threadfence();
-                    misc->merge_flag = last;
+                    misc->jobs[njob] = sg;
+                    ptx::mbar_arrive(bar(C::B_MJOB + njob));
+                }
+                ++njob;
+            }
+            ptx::tc_fence_before();
+        }
+        // merges of the row-blocks whose last piece this CTA wrote
+        for (int j = 0; ok && j < njob; ++j) {
+            ok = wait_bar(bar(C::B_MTICK + j), 0, wmisc, p);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            if (!misc->ticket[j]) continue;
+            __threadfence();
+            const Seg sg = misc->jobs[j];
+            const RB rb = rb_of(p, sg.w);
+            const long long tot = misc->span.tot;
+            const int c_first = cta_of(sg.pw, tot, NC);
+            const int c_last = cta_of(sg.pw + sg.ntiles - 1, tot, NC);
+            {
+                const bool c0_first = span_begin(c_first, tot, NC) == sg.pw;
+                const long long RW = BM * C::RBQ;
+                // slots of the CTAs that hold a piece of this row-block, compacted
+                if (warp == 0) {
+                    int nm = 0;
+                    for (int base = c_first; base <= c_last; base += 32) {
+                        const int cc = base + lane;
+                        const bool has = cc <= c_last && span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC);
+                        const unsigned m = __ballot_sync(0xffffffffu, has);
+                        const int k = nm + __popc(m & ((1u << lane) - 1u));
+                        if (has && k < kMaxMergeSlots) misc->mslot[k] = merge_slot(cc, c_first, c0_first);
+                        nm += __popc(m);
+                    }
+                    if (lane == 0) misc->nmerge = nm;
                 }
                 if (!xsync()) { ok = false; break; }
-                if (misc->merge_flag) {
-                    __threadfence();
-                    const bool c0_first = span_begin(c_first, tot, NC) == sg.pw;
-                    const long long RW = BM * C::RBQ;
+                const int nm = misc->nmerge;
+                if (nm <= kMaxMergeSlots) {
+                    // lse of each merged row: all partial lse loads issued together
+                    for (int r = stid; r < rb.rows_valid; r += NSOFT2) {
+                        const int hr = rb.g * p.G + (rb.qt * BM + r) / p.Tq;
+                        const float sk = (p.sink != nullptr) ? __ldg(p.sink + hr) : -INFINITY;
+                        float Lx = sk;
+                        float lv[8];
+                        for (int k0 = 0; k0 < nm; k0 += 8) {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                lv[j] = (k0 + j < nm) ? __ldcg(p.part_lse + misc->mslot[k0 + j] * RW + r) : -INFINITY;
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) Lx = fmaxf(Lx, lv[j]);
+                        }
+                        float lt = -INFINITY;
+                        if (Lx != -INFINITY) {
+                            float z = (sk != -INFINITY) ? __expf(sk - Lx) : 0.f;
+                            if (nm <= 8) {
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) z += __expf(lv[j] - Lx);
+                            } else {
+                                for (int k = 0; k < nm; ++k) z += __expf(__ldcg(p.part_lse + misc->mslot[k] * RW + r) - Lx);
+                            }
+                            lt = Lx + __logf(z);
+                        }
+                        misc->mlse[r] = lt;
+                        if (p.lse != nullptr) p.lse[rb.q_row0 + r] = lt;
+                    }
+                    if (!xsync()) { ok = false; break; }
+                    // O rows: weight exp(lse_k - lse) per piece; four pieces' loads in flight at once
+                    constexpr int C8 = C::D / 8;
+                    for (int it = stid; it < rb.rows_valid * C8; it += NSOFT2) {
+                        const int r = it / C8, c8 = it % C8;
+                        const float lt = misc->mlse[r];
+                        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        if (lt != -INFINITY) {
+                            for (int k0 = 0; k0 < nm; k0 += 4) {
+                                float lw[4];
+                                float4 xa[4], xb[4];
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    if (k0 + j < nm) {
+                                        const long long sl = misc->mslot[k0 + j];
+                                        const float4* src = reinterpret_cast<const float4*>(p.part_o + (sl * RW + r) * C::D + 8 * c8);
+                                        lw[j] = __ldcg(p.part_lse + sl * RW + r);
+                                        xa[j] = __ldcg(src);
+                                        xb[j] = __ldcg(src + 1);
+                                    } else {
+                                        lw[j] = -INFINITY;
+                                        xa[j] = xb[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                                    }
+                                }
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    const float wgt = __expf(lw[j] - lt);
+                                    acc[0] += wgt * xa[j].x; acc[1] += wgt * xa[j].y; acc[2] += wgt * xa[j].z; acc[3] += wgt * xa[j].w;
+                                    acc[4] += wgt * xb[j].x; acc[5] += wgt * xb[j].y; acc[6] += wgt * xb[j].z; acc[7] += wgt * xb[j].w;
+                                }
+                            }
+                        }
+                        *reinterpret_cast<uint4*>(p.out + (rb.q_row0 + r) * C::D + 8 * c8) =
+                            make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                       pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+                    }
+                } else {
+                    // more pieces than the slot list holds: walk the CTAs again
                     for (int r = stid; r < rb.rows_valid; r += NSOFT2) {
                         const int hr = rb.g * p.G + (rb.qt * BM + r) / p.Tq;
                         float Lx = (p.sink != nullptr) ? __ldg(p.sink + hr) : -INFINITY;
@@ -637,20 +775,19 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                 const long long sl = merge_slot(cc, c_first, c0_first);
                                 const float wgt = __expf(__ldcg(p.part_lse + sl * RW + r) - lt);
                                 const float4* src = reinterpret_cast<const float4*>(p.part_o + (sl * RW + r) * C::D + 8 * c8);
-                                const float4 a = __ldcg(src), b = __ldcg(src + 1);
-                                acc[0] += wgt * a.x; acc[1] += wgt * a.y; acc[2] += wgt * a.z; acc[3] += wgt * a.w;
-                                acc[4] += wgt * b.x; acc[5] += wgt * b.y; acc[6] += wgt * b.z; acc[7] += wgt * b.w;
+                                const float4 xa = __ldcg(src), xb = __ldcg(src + 1);
+                                acc[0] += wgt * xa.x; acc[1] += wgt * xa.y; acc[2] += wgt * xa.z; acc[3] += wgt * xa.w;
+                                acc[4] += wgt * xb.x; acc[5] += wgt * xb.y; acc[6] += wgt * xb.z; acc[7] += wgt * xb.w;
                             }
                         }
                         *reinterpret_cast<uint4*>(p.out + (rb.q_row0 + r) * C::D + 8 * c8) =
                             make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
                                        pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
                     }
-                    if (stid == 0) p.counters[sg.w] = 0;
                 }
-                if (!xsync()) { ok = false; break; }
+                if (stid == 0) p.counters[sg.w] = 0;
             }
-            ptx::tc_fence_before();
+            if (!xsync()) { ok = false; break; }
         }
     }
 
@@ -665,4 +802,4 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
 }  // namespace gqa
 
-static_assert(sizeof(gqa::Misc2) <= 2112, "misc block");
+static_assert(sizeof(gqa::Misc2) <= 2496, "misc block");

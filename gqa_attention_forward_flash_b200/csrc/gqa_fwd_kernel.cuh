@@ -166,12 +166,33 @@ struct SpanStart {
     int w, t;
 };
 
-// One full warp: total tiles, this CTA's span and the (row-block, tile) where it starts.
+// Tiles in one unit of a batch with logical length n (one thread).
+__device__ long long unit_tiles_thread(const Params& p, int n) {
+    if (!p.causal) {
+        int t = (n + p.BN - 1) / p.BN;
+        return static_cast<long long>(p.QW) * (t < 1 ? 1 : t);
+    }
+    long long acc = 0;
+    for (int qt = 0; qt < p.QW; ++qt) acc += qtile_ntiles(p, qt, n);
+    return acc;
+}
+
+// One full warp: total tiles, this CTA's span and the (row-block, tile) where it
+// starts.  With per-batch lengths and few row-blocks per unit every lane reads
+// its own batches' lengths, so the reads go out together (one memory round trip
+// for up to 32 batches), and the batch holding the span's first tile is found
+// with a warp scan and a ballot; with many row-blocks per unit (long causal
+// prefill) the lanes share each batch's row-blocks instead.
 __device__ void plan_span(const Params& p, int c, int NC, SpanStart* out) {
     const int lane = threadIdx.x & 31;
+    const bool lane_per_batch = !p.causal || p.QW <= 16;
     long long tot = 0;
     if (p.kv_lens == nullptr) {
         tot = static_cast<long long>(p.U) * unit_tiles_warp(p, p.Tkv);
+    } else if (lane_per_batch) {
+        long long mine = 0;
+        for (int b = lane; b < p.B; b += 32) mine += p.Hkv * unit_tiles_thread(p, load_len(p, b));
+        tot = warp_sum_ll(mine);
     } else {
         for (int b = 0; b < p.B; ++b) tot += p.Hkv * unit_tiles_warp(p, load_len(p, b));
     }
@@ -185,12 +206,36 @@ __device__ void plan_span(const Params& p, int c, int NC, SpanStart* out) {
             per_unit = unit_tiles_warp(p, n);
             b = static_cast<int>(p0 / (per_unit * p.Hkv));
             acc = static_cast<long long>(b) * per_unit * p.Hkv;
-        } else {
+        } else if (!lane_per_batch) {
             for (b = 0; b < p.B; ++b) {
                 n = load_len(p, b);
                 per_unit = unit_tiles_warp(p, n);
                 if (p0 < acc + per_unit * p.Hkv) break;
                 acc += per_unit * p.Hkv;
+            }
+        } else {
+            for (int base = 0; base < p.B; base += 32) {
+                const int bb = base + lane;
+                const int nb = bb < p.B ? load_len(p, bb) : 0;
+                const long long ub = bb < p.B ? unit_tiles_thread(p, nb) : 0;
+                const long long cnt = ub * p.Hkv;
+                long long inc = cnt;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const long long y = __shfl_up_sync(0xffffffffu, inc, o);
+                    if (lane >= o) inc += y;
+                }
+                const long long chunk_total = __shfl_sync(0xffffffffu, inc, 31);
+                if (p0 < acc + chunk_total) {
+                    const unsigned hit = __ballot_sync(0xffffffffu, p0 < acc + inc);
+                    const int L = __ffs(hit) - 1;
+                    b = base + L;
+                    n = __shfl_sync(0xffffffffu, nb, L);
+                    per_unit = __shfl_sync(0xffffffffu, ub, L);
+                    acc += __shfl_sync(0xffffffffu, inc - cnt, L);
+                    break;
+                }
+                acc += chunk_total;
             }
         }
         const long long in_b = p0 - acc;
