@@ -163,7 +163,8 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tmem = misc->tmem_base;
 
     if (warp >= 8) {
-        ptx::regs_dec<64>();
+        // 128 x 88 + 256 x 208 = 384 x 168, the registers the block is launched with
+        ptx::regs_dec<88>();
         // ------------------------------------------------------------ producers
         if (warp == 8 && lane == 0) {
             const uint64_t pol_q = ptx::policy_evict_last();
