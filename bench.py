@@ -342,7 +342,7 @@ def run_ours(args, w, ws, rank, local):
     traffic = traffic_for(w)
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": traffic, "peak_source": peak_src + (" (burst)" if bound == "tensor" else ""),
-                "kernel": main_kernel_name(w), "kernel_ms": main_avg, "launches_per_step": 1,
+                "kernel": main_kernel_name(w), "kernel_ms": main_avg, "launches_per_step": launches_per_call(w),
                 "algorithmic_bytes": nbytes, "algorithmic_flops": nflops}
 
     # end to end through the public API with host buffers
@@ -360,7 +360,7 @@ def run_ours(args, w, ws, rank, local):
             "metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(w),
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": len(main_ms),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": len(main_ms) * launches_per_call(w),
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -412,8 +412,13 @@ def run_e2e(args, w, inp, dev, stream, nbytes, nflops, ws):
 
 
 def main_kernel_name(w: Workload) -> str:
-    """The kernel gqa_attention_fwd launches for this head dim (its only launch)."""
-    return "gqa_fwd2_kernel" if w.d <= 128 else "gqa_fwd_kernel"
+    """The kernel(s) gqa_attention_fwd launches for this head dim."""
+    return "gqa_fwd2_kernel" if w.d <= 128 else "gqa_fwd_kernel + gqa_combine_streamk_kernel"
+
+
+def launches_per_call(w: Workload) -> int:
+    """Head dims 64/128 merge split rows inside the one kernel; 256/512 add the combine kernel."""
+    return 1 if w.d <= 128 else 2
 
 
 def kernel_source_digest() -> str:

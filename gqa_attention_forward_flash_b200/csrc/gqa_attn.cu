@@ -153,6 +153,16 @@ using Cfg512 = FwdCfg<512, 32, 2, 2, 1, 2>;
 
 int dsplit_for(int d) { return d == 512 ? Cfg512::DSPLIT : 1; }
 
+// Head dims served by the single-lane kernel merge their split row-blocks in a
+// second kernel spread over every SM (their partial rows are long: 256 or 512
+// columns, up to one piece per CTA group); the two-lane kernel merges in place.
+bool uses_combine_kernel(int d) { return d == 256 || d == 512; }
+
+int launch_streamk_combine(const Params& p, int ds, int sm_count, cudaStream_t st) {
+    gqa_combine_streamk_kernel<<<2 * sm_count, 256, 0, st>>>(p, ds, BM * p.RBQ);
+    return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
 // Tile geometry of the kernel that will serve these sizes.
 void choose_geometry(Params& p) {
     if (p.d == 512) {
@@ -301,16 +311,19 @@ extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, co
     if (NC < 1) NC = 1;
     const size_t slot_rows = static_cast<size_t>(2 * NC) * ds * BM * p.RBQ;
     const size_t slot_o = slot_rows * (d / ds) * sizeof(float);
-    const size_t slot_l = slot_rows * sizeof(float);
-    rc = ensure_scratch(*s, slot_o + slot_l);
+    const size_t slot_l = (slot_rows * sizeof(float) + 255) & ~static_cast<size_t>(255);
+    const size_t jobs = static_cast<size_t>(p.W) * ds * sizeof(CJob);
+    rc = ensure_scratch(*s, slot_o + slot_l + jobs);
     if (rc) return rc;
-    rc = ensure_counters(*s, p.W * ds);
+    rc = ensure_counters(*s, p.W * ds + 2);
     if (rc) return rc;
     char* base = static_cast<char*>(s->scratch);
     p.mode = 0;
     p.part_o = reinterpret_cast<float*>(base);
     p.part_lse = reinterpret_cast<float*>(base + slot_o);
+    p.cjobs = reinterpret_cast<CJob*>(base + slot_o + slot_l);
     p.counters = s->counters;
+    p.cjob_count = s->counters + p.W * ds;
     p.err = s->err;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaEvent_t* ev = nullptr;
@@ -319,8 +332,14 @@ extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, co
         cudaGetDevice(&dev);
         if (dev == g_prof.dev) ev = g_prof.ev[g_prof.n++];
     }
-    rc = dispatch_fwd(p, q, k, v, NC * ds, st, ev ? ev[0] : nullptr, ev ? ev[1] : nullptr);
+    const bool combine = uses_combine_kernel(d);
+    rc = dispatch_fwd(p, q, k, v, NC * ds, st, ev ? ev[0] : nullptr, (ev && !combine) ? ev[1] : nullptr);
     if (rc) return rc;
+    if (combine) {
+        rc = launch_streamk_combine(p, ds, s->sm_count, st);
+        if (rc) return rc;
+        if (ev && cudaEventRecord(ev[1], st) != cudaSuccess) return GQA_ERR_CUDA;
+    }
     return GQA_OK;
 }
 
@@ -461,11 +480,13 @@ namespace {
 
 constexpr size_t kNaCounterInts = 65536;                         // merge tickets: at most this many row-blocks
 constexpr size_t kNaErrOffset = kNaCounterInts * sizeof(int);    // device error word
+constexpr size_t kNaJobCountOffset = kNaErrOffset + 16;           // combine jobs listed / blocks done
 constexpr size_t kNaLseOffset = kNaErrOffset + 256;
 constexpr size_t kNaLseFloats = static_cast<size_t>(2) * kMaxCtas * 2 * BM;  // 2 slots x 256 rows per CTA
 constexpr size_t kNaPartOffset = kNaLseOffset + kNaLseFloats * sizeof(float);
 constexpr size_t kNaPartBytes = static_cast<size_t>(20) << 20;  // fp32 partial O: 20 MiB
-constexpr size_t kNaBytes = kNaPartOffset + kNaPartBytes;       // about 21.3 MiB in all
+constexpr size_t kNaJobsOffset = kNaPartOffset + kNaPartBytes;  // combine jobs: one per row-block at most
+constexpr size_t kNaBytes = kNaJobsOffset + kNaCounterInts * sizeof(CJob);  // about 23.3 MiB in all
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNaBytes];
 
@@ -554,10 +575,15 @@ extern "C" int gqa_attention_fwd_noalloc(const void* q, const void* k, const voi
     p.part_lse = reinterpret_cast<float*>(base + kNaLseOffset);
     p.counters = reinterpret_cast<int*>(base);
     p.err = reinterpret_cast<int*>(base + kNaErrOffset);
+    p.cjobs = reinterpret_cast<CJob*>(base + kNaJobsOffset);
+    p.cjob_count = reinterpret_cast<int*>(base + kNaJobCountOffset);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // the array keeps the last call's contents: the merge tickets and the error
-    // word must start at zero
+    // the array keeps the last call's contents: the merge tickets, the error word
+    // and the combine-job counters must start at zero
     if (cudaMemsetAsync(base, 0, static_cast<size_t>(p.W) * sizeof(int), st) != cudaSuccess) return GQA_ERR_CUDA;
-    if (cudaMemsetAsync(base + kNaErrOffset, 0, sizeof(int), st) != cudaSuccess) return GQA_ERR_CUDA;
-    return dispatch_fwd(p, q, k, v, static_cast<int>(NC), st);
+    if (cudaMemsetAsync(base + kNaErrOffset, 0, 32, st) != cudaSuccess) return GQA_ERR_CUDA;
+    rc = dispatch_fwd(p, q, k, v, static_cast<int>(NC), st);
+    if (rc) return rc;
+    if (uses_combine_kernel(d)) return launch_streamk_combine(p, 1, s->sm_count, st);
+    return GQA_OK;
 }

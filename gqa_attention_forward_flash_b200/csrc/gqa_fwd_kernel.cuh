@@ -51,11 +51,23 @@ constexpr int NSOFT = 256;       // softmax threads
 constexpr int NSOFT_WARPS = NSOFT / 32;  // arrivals per softmax-side barrier phase (one per warp)
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
-constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
+constexpr float RESCALE_THRESHOLD = 8.0f;
+constexpr int kMaxCombinePieces = 512;  // CTA groups of a split (the grid is at most 512 CTAs)  // log2 units: rescale O only when the max grows by > 2^8
 
 // device error codes (same values as gqa_status)
 constexpr int DEV_ERR_TIMEOUT = -6;
 constexpr int DEV_ERR_KVLEN = -8;
+
+// A split row-block (one DSPLIT part of its O columns) whose pieces are all
+// written: the stream-K combine kernel merges it.
+struct CJob {
+    long long pw;   // flat index of the row-block's first tile
+    long long tot;  // tiles of the whole problem (the stream-K split)
+    int w;          // row-block
+    int ntiles;     // its key tiles
+    int ho;         // which DSPLIT part of the O columns
+    int nc;         // CTA groups of the split
+};
 
 struct Params {
     int B, Hq, Hkv, Tq, Tkv, d;
@@ -81,6 +93,8 @@ struct Params {
     int spread;           // 1: packed row r lives in TMEM lane (r / rq) * 32 + r % rq (R <= 96)
     int rq;               // packed rows per lane quadrant in the spread layout
     int kv_box_rows;      // rows of one K/V TMA box: min(BN, B*Hkv*Tkv)
+    CJob* cjobs;          // single-lane kernel, mode 0: [W*DSPLIT] row-blocks for the combine kernel
+    int* cjob_count;      // [2]: jobs listed, combine blocks done (zero between calls)
 };
 
 // ------------------------------------------------------------------ schedule
@@ -947,8 +961,9 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (valid && half == 0 && (sg.kind == 1 || ho == 0)) __stcg(dl, lse_v);
 
                 if (sg.kind == 1) {
-                    __threadfence();  // this thread's partial rows are visible before the ticket
-                    // ---- ticket: the last CTA to finish a piece of this row-block merges
+                    // ---- ticket: the CTA that completes the row-block's pieces lists it for the
+                    // stream-K combine kernel, which merges every listed row-block across all SMs
+                    // (it runs after this kernel, so the partial rows need no fence here)
                     const long long tot = misc->span.tot;
                     const int c_first = cta_of(sg.pw, tot, NC);
                     const int c_last = cta_of(sg.pw + sg.ntiles - 1, tot, NC);
@@ -957,62 +972,19 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         int ncontrib = 0;
                         for (int cc = c_first; cc <= c_last; ++cc)
                             ncontrib += span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC);
-                        __threadfence();
-                        const int old = atomicAdd(p.counters + static_cast<long long>(sg.w) * C::DSPLIT + ho, 1);
-                        const int last = (old == ncontrib - 1);
-                        if (last) __threadfence();
-                        misc->merge_flag = last;
-                    }
-                    if (!xsync()) { ok = false; break; }
-                    if (misc->merge_flag) {
-                        __threadfence();
-                        const bool c0_first = span_begin(c_first, tot, NC) == sg.pw;
-                        // merged lse per packed row
-                        for (int r = stid; r < rb.rows_valid; r += NSOFT) {
-                            const int hr = rb.g * p.G + (rb.qt * BM + r) / p.Tq;
-                            float L = (p.sink != nullptr) ? __ldg(p.sink + hr) : -INFINITY;
-                            for (int cc = c_first; cc <= c_last; ++cc) {
-                                if (!(span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC))) continue;
-                                const long long sl = merge_slot(cc, c_first, c0_first) * C::DSPLIT + ho;
-                                L = fmaxf(L, __ldcg(p.part_lse + sl * BM + r));
-                            }
-                            float lt = -INFINITY;
-                            if (L != -INFINITY) {
-                                float z = (p.sink != nullptr) ? __expf(__ldg(p.sink + hr) - L) : 0.f;
-                                for (int cc = c_first; cc <= c_last; ++cc) {
-                                    if (!(span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC))) continue;
-                                    const long long sl = merge_slot(cc, c_first, c0_first) * C::DSPLIT + ho;
-                                    z += __expf(__ldcg(p.part_lse + sl * BM + r) - L);
-                                }
-                                lt = L + __logf(z);
-                            }
-                            misc->mlse[r] = lt;
-                            if (p.lse != nullptr && ho == 0) p.lse[rb.q_row0 + r] = lt;
+                        const long long ctr = static_cast<long long>(sg.w) * C::DSPLIT + ho;
+                        const int old = atomicAdd(p.counters + ctr, 1);
+                        if (old == ncontrib - 1) {
+                            p.counters[ctr] = 0;  // ready for the next call
+                            CJob jb;
+                            jb.pw = sg.pw;
+                            jb.tot = tot;
+                            jb.w = sg.w;
+                            jb.ntiles = sg.ntiles;
+                            jb.ho = ho;
+                            jb.nc = NC;
+                            p.cjobs[atomicAdd(p.cjob_count, 1)] = jb;
                         }
-                        if (!xsync()) { ok = false; break; }
-                        // weighted sum of the partials, 8 columns per item
-                        constexpr int C8 = C::DO / 8;
-                        for (int it = stid; it < rb.rows_valid * C8; it += NSOFT) {
-                            const int r = it / C8, c8 = it % C8;
-                            const float lt = misc->mlse[r];
-                            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                            if (lt != -INFINITY) {
-                                for (int cc = c_first; cc <= c_last; ++cc) {
-                                    if (!(span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC))) continue;
-                                    const long long sl = merge_slot(cc, c_first, c0_first) * C::DSPLIT + ho;
-                                    const float wgt = __expf(__ldcg(p.part_lse + sl * BM + r) - lt);
-                                    const float4* src =
-                                        reinterpret_cast<const float4*>(p.part_o + (sl * BM + r) * C::DO + 8 * c8);
-                                    const float4 a = __ldcg(src), b = __ldcg(src + 1);
-                                    acc[0] += wgt * a.x; acc[1] += wgt * a.y; acc[2] += wgt * a.z; acc[3] += wgt * a.w;
-                                    acc[4] += wgt * b.x; acc[5] += wgt * b.y; acc[6] += wgt * b.z; acc[7] += wgt * b.w;
-                                }
-                            }
-                            *reinterpret_cast<uint4*>(p.out + (rb.q_row0 + r) * C::D + ho * C::DO + 8 * c8) =
-                                make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                                           pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
-                        }
-                        if (stid == 0) p.counters[static_cast<long long>(sg.w) * C::DSPLIT + ho] = 0;  // ready for the next call
                     }
                 }
             }
@@ -1034,6 +1006,118 @@ gqa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 // ------------------------------------------------------------------ public combine kernel
 
 // Uniform combine (public entry): one warp per row, S partials laid out [rows, S, d].
+// Stream-K combine (single-lane kernel, mode 0): merges the row-blocks the main
+// kernel listed, each from its pieces' partial (O, lse) in the slots 2c / 2c + 1 of
+// the CTA groups c that hold a piece, into O (bf16) and lse:
+//   lse = log(e^sink + sum_k e^lse_k),  O = sum_k e^(lse_k - lse) O_k.
+// A block takes 8 rows of one listed row-block at a time (grid-stride over all of
+// them): one warp per row finds its lse and the pieces' weights, then every
+// thread sums 8 columns of a row over the pieces, four pieces' loads at a time.
+// The last block to finish leaves the job counter at zero for the next call.
+constexpr int kCombRows = 8;
+__global__ void __launch_bounds__(256)
+gqa_combine_streamk_kernel(const Params p, int dsplit, int rw) {
+    __shared__ int slot_s[kMaxCombinePieces];
+    __shared__ float wgt_s[kCombRows][kMaxCombinePieces];
+    __shared__ float lse_s[kCombRows];
+    __shared__ int npieces_s;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int njobs = *reinterpret_cast<volatile int*>(p.cjob_count);
+    const int DO = p.d / dsplit;
+    const int chunks = (rw + kCombRows - 1) / kCombRows;
+    const long long units = static_cast<long long>(njobs) * chunks;
+    for (long long u = blockIdx.x; u < units; u += gridDim.x) {
+        const CJob jb = p.cjobs[u / chunks];
+        const int r0 = static_cast<int>(u % chunks) * kCombRows;
+        const RB rb = rb_of(p, jb.w);
+        const int nrows = min(kCombRows, rb.rows_valid - r0);
+        if (nrows <= 0) continue;
+        const int c_first = cta_of(jb.pw, jb.tot, jb.nc);
+        const int c_last = cta_of(jb.pw + jb.ntiles - 1, jb.tot, jb.nc);
+        const bool c0_first = span_begin(c_first, jb.tot, jb.nc) == jb.pw;
+        if (warp == 0) {
+            int nm = 0;
+            for (int base = c_first; base <= c_last; base += 32) {
+                const int cc = base + lane;
+                const bool has = cc <= c_last && span_begin(cc, jb.tot, jb.nc) < span_begin(cc + 1, jb.tot, jb.nc);
+                const unsigned m = __ballot_sync(0xffffffffu, has);
+                const int k = nm + __popc(m & ((1u << lane) - 1u));
+                if (has && k < kMaxCombinePieces)
+                    slot_s[k] = static_cast<int>(merge_slot(cc, c_first, c0_first) * dsplit + jb.ho);
+                nm += __popc(m);
+            }
+            if (lane == 0) npieces_s = nm < kMaxCombinePieces ? nm : kMaxCombinePieces;
+        }
+        __syncthreads();
+        const int np = npieces_s;
+        // lse and the pieces' weights of each row: one warp per row
+        if (warp < nrows) {
+            const int r = r0 + warp;
+            const int hr = rb.g * p.G + (rb.qt * BM + r) / p.Tq;
+            const float sk = (p.sink != nullptr) ? __ldg(p.sink + hr) : -INFINITY;
+            float mx = sk;
+            for (int k = lane; k < np; k += 32) mx = fmaxf(mx, __ldcg(p.part_lse + static_cast<long long>(slot_s[k]) * rw + r));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            float z = 0.f;
+            if (mx != -INFINITY) {
+                for (int k = lane; k < np; k += 32) z += __expf(__ldcg(p.part_lse + static_cast<long long>(slot_s[k]) * rw + r) - mx);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+                if (sk != -INFINITY) z += __expf(sk - mx);
+            }
+            const float lt = (mx != -INFINITY && z > 0.f) ? mx + __logf(z) : -INFINITY;
+            for (int k = lane; k < np; k += 32)
+                wgt_s[warp][k] = (lt != -INFINITY) ? __expf(__ldcg(p.part_lse + static_cast<long long>(slot_s[k]) * rw + r) - lt) : 0.f;
+            if (lane == 0) {
+                lse_s[warp] = lt;
+                if (p.lse != nullptr && jb.ho == 0) p.lse[rb.q_row0 + r] = lt;
+            }
+        }
+        __syncthreads();
+        // O: 8 columns per item
+        const int C8 = DO / 8;
+        for (int it = threadIdx.x; it < nrows * C8; it += blockDim.x) {
+            const int rr = it / C8, c8 = it % C8;
+            const int r = r0 + rr;
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int k0 = 0; k0 < np; k0 += 4) {
+                float4 xa[4], xb[4];
+                float wk[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (k0 + j < np) {
+                        const float4* src = reinterpret_cast<const float4*>(
+                            p.part_o + (static_cast<long long>(slot_s[k0 + j]) * rw + r) * DO + 8 * c8);
+                        xa[j] = __ldcg(src);
+                        xb[j] = __ldcg(src + 1);
+                        wk[j] = wgt_s[rr][k0 + j];
+                    } else {
+                        xa[j] = xb[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        wk[j] = 0.f;
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc[0] += wk[j] * xa[j].x; acc[1] += wk[j] * xa[j].y; acc[2] += wk[j] * xa[j].z; acc[3] += wk[j] * xa[j].w;
+                    acc[4] += wk[j] * xb[j].x; acc[5] += wk[j] * xb[j].y; acc[6] += wk[j] * xb[j].z; acc[7] += wk[j] * xb[j].w;
+                }
+            }
+            *reinterpret_cast<uint4*>(p.out + (rb.q_row0 + r) * p.d + jb.ho * DO + 8 * c8) =
+                make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                           pack_bf16x2(acc[6], acc[7]));
+        }
+        __syncthreads();  // slot_s / wgt_s are rewritten by the next unit
+    }
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(p.cjob_count + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+            p.cjob_count[0] = 0;
+            p.cjob_count[1] = 0;
+        }
+    }
+}
+
 __global__ void __launch_bounds__(256)
 gqa_combine_uniform_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part, int S,
                            const float* __restrict__ sink, __nv_bfloat16* __restrict__ out,
