@@ -1019,7 +1019,6 @@ __global__ void __launch_bounds__(256)
 gqa_combine_streamk_kernel(const Params p, int dsplit, int rw) {
     __shared__ int slot_s[kMaxCombinePieces];
     __shared__ float wgt_s[kCombRows][kMaxCombinePieces];
-    __shared__ float lse_s[kCombRows];
     __shared__ int npieces_s;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int njobs = *reinterpret_cast<volatile int*>(p.cjob_count);
@@ -1069,10 +1068,7 @@ gqa_combine_streamk_kernel(const Params p, int dsplit, int rw) {
             const float lt = (mx != -INFINITY && z > 0.f) ? mx + __logf(z) : -INFINITY;
             for (int k = lane; k < np; k += 32)
                 wgt_s[warp][k] = (lt != -INFINITY) ? __expf(__ldcg(p.part_lse + static_cast<long long>(slot_s[k]) * rw + r) - lt) : 0.f;
-            if (lane == 0) {
-                lse_s[warp] = lt;
-                if (p.lse != nullptr && jb.ho == 0) p.lse[rb.q_row0 + r] = lt;
-            }
+            if (lane == 0 && p.lse != nullptr && jb.ho == 0) p.lse[rb.q_row0 + r] = lt;
         }
         __syncthreads();
         // O: 8 columns per item
