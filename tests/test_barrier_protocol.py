@@ -1,0 +1,354 @@
+"""CPU model of the kernels' mbarrier protocol (host logic; no GPU).
+
+Every role of a CTA (Q/K producer, V producer, MMA issuer, softmax warps, the
+ticket warp) is written as a generator of the waits, arrivals and asynchronous
+completions its code performs, in the same order and with the same phase
+arithmetic.  A random scheduler interleaves the roles; TMA loads complete in
+any order, MMA commits in issue order (one thread's tcgen05 MMAs execute in
+order).  Two properties are checked on many random segment layouts:
+
+* no deadlock: some role can always move until all have finished;
+* no phase aliasing: when a role waits for completion k of a barrier, the
+  barrier has never completed k + 2 or more phases (an mbarrier parity wait
+  cannot tell phase k from k + 2, so such a wait would hang or pass wrongly).
+
+A planted protocol error (an off-by-one wait index) must be caught.
+"""
+import random
+
+import pytest
+
+
+class _Bar:
+    def __init__(self, count):
+        self.count, self.arrived, self.done = count, 0, 0
+
+    def arrive(self):
+        self.arrived += 1
+        if self.arrived == self.count:
+            self.arrived = 0
+            self.done += 1
+
+
+class ProtocolError(RuntimeError):
+    pass
+
+
+def _simulate(bars, roles, rnd):
+    """roles: name -> generator of ('wait', bar, k) | ('arrive', bar) | ('mma', [bars]) | ('tma', [bars])."""
+    state = {r: None for r in roles}
+    mma_q, tma_q = [], []
+    while roles:
+        runnable = []
+        for r in roles:
+            st = state[r]
+            if st is None:
+                runnable.append(r)
+                continue
+            b = bars[st[1]]
+            if b.done > st[2] + 1:
+                raise ProtocolError("aliasing: %s waits for completion %d of %s, %d done" % (r, st[2], st[1], b.done))
+            if b.done > st[2]:
+                runnable.append(r)
+        choices = runnable + (["<mma done>"] if mma_q else []) + (["<tma done>"] if tma_q else [])
+        if not choices:
+            raise ProtocolError("deadlock: " + ", ".join("%s@%s" % (r, state[r][1:]) for r in roles))
+        c = rnd.choice(choices)
+        if c == "<mma done>":
+            for b in mma_q.pop(0):
+                bars[b].arrive()
+            continue
+        if c == "<tma done>":
+            for b in tma_q.pop(rnd.randrange(len(tma_q))):
+                bars[b].arrive()
+            continue
+        state[c] = None
+        try:
+            op = next(roles[c])
+        except StopIteration:
+            del roles[c], state[c]
+            continue
+        if op[0] == "wait":
+            if op[2] >= 0:
+                state[c] = op
+        elif op[0] == "arrive":
+            bars[op[1]].arrive()
+        elif op[0] == "mma":
+            mma_q.append(op[1])
+        elif op[0] == "tma":
+            tma_q.append(op[1])
+
+
+# --------------------------------------------------------------------------
+# two-lane kernel (head dims 64 / 128): gqa_fwd2_kernel
+
+
+def _two_lane(segs, rbq, stk, stv, rnd, mutate=False):
+    """segs: list of (ntiles, kind); kind 1 = split segment (partial rows + ticket)."""
+    bars = {}
+
+    def mk(name, count):
+        bars[name] = _Bar(count)
+
+    mk("QFULL", 1)
+    mk("QEMPTY", 1)
+    for i in range(stk):
+        mk("KF%d" % i, 1)
+        mk("KE%d" % i, 1)
+    for i in range(stv):
+        mk("VF%d" % i, 1)
+        mk("VE%d" % i, 1)
+    for lane in range(2):
+        mk("SF%d" % lane, 1)
+        mk("PF%d" % lane, 4)
+        mk("OD%d" % lane, 1)
+    mk("X", 8)
+    for j in range(2):
+        mk("MJ%d" % j, 1)
+        mk("MT%d" % j, 1)
+    tail = [[rnd.random() < 0.3 for _ in range(n)] for n, _ in segs]
+    merges = [rnd.random() < 0.5 for _ in segs]
+    nsplit = min(2, sum(1 for _, k in segs if k == 1))
+
+    def kprod():
+        g = 0
+        for si, (n, _) in enumerate(segs):
+            yield ("wait", "QEMPTY", si - 1)
+            yield ("tma", ["QFULL"])
+            for _ in range(n):
+                yield ("wait", "KE%d" % (g % stk), g // stk - 1)
+                yield ("tma", ["KF%d" % (g % stk)])
+                g += 1
+
+    def vprod():
+        g = 0
+        for n, _ in segs:
+            for _ in range(n):
+                yield ("wait", "VE%d" % (g % stv), g // stv - 1)
+                yield ("tma", ["VF%d" % (g % stv)])
+                g += 1
+
+    def mma():
+        g = 0
+        n_pv = [0, 0]
+
+        def pv(lane, gv, wait_v):
+            idx = n_pv[lane] + (1 if mutate else 0)
+            yield ("wait", "PF%d" % lane, idx)
+            n_pv[lane] += 1
+            if wait_v:
+                yield ("wait", "VF%d" % (gv % stv), gv // stv)
+            yield ("mma", ["OD%d" % lane, "VE%d" % (gv % stv)] if rbq == 1 or lane == 1 else ["OD%d" % lane])
+
+        for si, (n, _) in enumerate(segs):
+            yield ("wait", "QFULL", si)
+            prev = None
+            pend_b = None
+            for t in range(n):
+                yield ("wait", "KF%d" % (g % stk), g // stk)
+                last = ["QEMPTY"] if t == n - 1 else []
+                if rbq == 1:
+                    lane = g & 1
+                    yield ("mma", ["SF%d" % lane, "KE%d" % (g % stk)] + last)
+                    if prev is not None:
+                        yield from pv(prev[0], prev[1], True)
+                    prev = (lane, g)
+                else:
+                    yield ("mma", ["SF0"])
+                    if pend_b is not None:
+                        yield from pv(1, pend_b, False)
+                    yield ("mma", ["SF1", "KE%d" % (g % stk)] + last)
+                    yield from pv(0, g, True)
+                    pend_b = g
+                g += 1
+            # the segment's last PV goes out when its tile loop ends
+            if prev is not None:
+                yield from pv(prev[0], prev[1], True)
+            if pend_b is not None:
+                yield from pv(1, pend_b, False)
+
+    xph = [0] * 8
+
+    def softmax(w):
+        lane = w // 4
+        g = 0
+        cnt = 0
+        njob = 0
+
+        def xsync():
+            yield ("arrive", "X")
+            yield ("wait", "X", xph[w])
+            xph[w] += 1
+
+        for si, (n, kind) in enumerate(segs):
+            mine = 0
+            for t in range(n):
+                if rbq == 1 and (g & 1) != lane:
+                    g += 1
+                    continue
+                yield ("wait", "SF%d" % lane, cnt)
+                if mine > 0 and rnd.random() < 0.3:  # lazy rescale (decided per warp)
+                    yield ("wait", "OD%d" % lane, cnt - 1)
+                if tail[si][t]:  # zeroing padded V rows of the tile
+                    yield ("wait", "VF%d" % (g % stv), g // stv)
+                yield ("arrive", "PF%d" % lane)
+                cnt += 1
+                mine += 1
+                g += 1
+            if mine > 0:
+                yield ("wait", "OD%d" % lane, cnt - 1)
+            if rbq == 1:
+                yield from xsync()
+            yield from xsync()
+            if kind == 1 and njob < 2:
+                if w == 0:
+                    yield ("arrive", "MJ%d" % njob)
+                njob += 1
+        for j in range(njob):
+            yield ("wait", "MT%d" % j, 0)
+            if merges[j]:
+                for _ in range(3):
+                    yield from xsync()
+
+    def tickets():
+        for j in range(nsplit):
+            yield ("wait", "MJ%d" % j, 0)
+            yield ("arrive", "MT%d" % j)
+
+    roles = {"kprod": kprod(), "vprod": vprod(), "mma": mma(), "tickets": tickets()}
+    for w in range(8):
+        roles["softmax%d" % w] = softmax(w)
+    _simulate(bars, roles, rnd)
+
+
+# --------------------------------------------------------------------------
+# single-lane kernel (head dims 256 / 512): gqa_fwd_kernel
+
+
+def _single_lane(segs, stk, stv, rnd):
+    bars = {}
+
+    def mk(name, count):
+        bars[name] = _Bar(count)
+
+    mk("QFULL", 1)
+    mk("QEMPTY", 1)
+    for i in range(stk):
+        mk("KF%d" % i, 1)
+        mk("KE%d" % i, 1)
+    for i in range(stv):
+        mk("VF%d" % i, 1)
+        mk("VE%d" % i, 1)
+    for b in range(2):
+        mk("SF%d" % b, 1)
+        mk("SR%d" % b, 8)
+        mk("PF%d" % b, 8)
+        mk("OD%d" % b, 1)
+    mk("X", 8)
+    tail = [[rnd.random() < 0.3 for _ in range(n)] for n, _ in segs]
+
+    def kprod():
+        g = 0
+        for si, (n, _) in enumerate(segs):
+            yield ("wait", "QEMPTY", si - 1)
+            yield ("tma", ["QFULL"])
+            for _ in range(n):
+                yield ("wait", "KE%d" % (g % stk), g // stk - 1)
+                yield ("tma", ["KF%d" % (g % stk)])
+                g += 1
+
+    def vprod():
+        g = 0
+        for n, _ in segs:
+            for _ in range(n):
+                yield ("wait", "VE%d" % (g % stv), g // stv - 1)
+                yield ("tma", ["VF%d" % (g % stv)])
+                g += 1
+
+    def mma():
+        g = 0
+        prev = None
+
+        def pv(gp):
+            pb = gp & 1
+            yield ("wait", "PF%d" % pb, gp >> 1)
+            yield ("wait", "VF%d" % (gp % stv), gp // stv)
+            yield ("mma", ["OD%d" % pb, "VE%d" % (gp % stv)])
+
+        for si, (n, _) in enumerate(segs):
+            yield ("wait", "QFULL", si)
+            for t in range(n):
+                sb = g & 1
+                yield ("wait", "KF%d" % (g % stk), g // stk)
+                if g >= 2:
+                    yield ("wait", "SR%d" % sb, (g >> 1) - 1)
+                yield ("mma", ["SF%d" % sb, "KE%d" % (g % stk)] + (["QEMPTY"] if t == n - 1 else []))
+                if prev is not None:
+                    yield from pv(prev)
+                prev = g
+                g += 1
+        if prev is not None:
+            yield from pv(prev)
+
+    xph = [0] * 8
+
+    def softmax(w):
+        g = 0
+
+        def xsync():
+            yield ("arrive", "X")
+            yield ("wait", "X", xph[w])
+            xph[w] += 1
+
+        for si, (n, kind) in enumerate(segs):
+            for t in range(n):
+                sb = g & 1
+                yield ("wait", "SF%d" % sb, g >> 1)
+                yield ("arrive", "SR%d" % sb)
+                if g >= 2:
+                    yield ("wait", "OD%d" % sb, (g >> 1) - 1)
+                if t > 0 and rnd.random() < 0.3:
+                    yield ("wait", "OD%d" % ((g - 1) & 1), (g - 1) >> 1)
+                if tail[si][t]:
+                    yield ("wait", "VF%d" % (g % stv), g // stv)
+                yield ("arrive", "PF%d" % sb)
+                g += 1
+            yield from xsync()
+            if n > 0:
+                yield ("wait", "OD%d" % ((g - 1) & 1), (g - 1) >> 1)
+            if kind == 1:
+                yield from xsync()
+            yield from xsync()
+
+    roles = {"kprod": kprod(), "vprod": vprod(), "mma": mma()}
+    for w in range(8):
+        roles["softmax%d" % w] = softmax(w)
+    _simulate(bars, roles, rnd)
+
+
+def _layouts(seed, count):
+    rnd = random.Random(seed)
+    for trial in range(count):
+        segs = [(rnd.randint(1, 6), rnd.choice([0, 1])) for _ in range(rnd.randint(1, 5))]
+        yield trial, segs, rnd.randint(2, 4), rnd.randint(2, 4)
+
+
+@pytest.mark.parametrize("rbq", [1, 2])
+def test_two_lane_protocol_has_no_deadlock_or_aliasing(rbq):
+    for trial, segs, stk, stv in _layouts(11 + rbq, 400):
+        _two_lane(segs, rbq, stk, stv, random.Random(trial))
+
+
+def test_single_lane_protocol_has_no_deadlock_or_aliasing():
+    for trial, segs, stk, stv in _layouts(7, 400):
+        _single_lane(segs, stk, stv, random.Random(trial))
+
+
+def test_model_catches_a_wrong_wait_index():
+    caught = 0
+    for trial, segs, stk, stv in _layouts(3, 60):
+        try:
+            _two_lane(segs, 1, stk, stv, random.Random(trial), mutate=True)
+        except ProtocolError:
+            caught += 1
+    assert caught == 60
