@@ -36,7 +36,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from gqa_attention_forward_flash_b200.synth import WORKLOADS, Workload, make_inputs  # noqa: E402
+from gqa_attention_forward_flash_b200.synth import WORKLOADS, Workload, make_inputs, paginate  # noqa: E402
 
 METRIC = "GQA fwd TFLOP/s (prefill) & KV HBM GB/s (decode), 1 B200, % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -257,7 +257,7 @@ def run_reference(args, w, ws, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * statistics.mean(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_of(w),
+        "data": "synthetic", "config": config_of(w, args.page_size),
         "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
                          "sample": "per step: " + desc},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -265,13 +265,21 @@ def run_reference(args, w, ws, rank):
     print(json.dumps(line), flush=True)
 
 
-def config_of(w: Workload):
+def config_of(w: Workload, page_size: int = 0):
     c = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "G": w.G, "Tq": w.Tq, "Tkv": w.Tkv, "d": w.d,
          "causal": w.causal, "sink": w.sink, "seed": w.seed,
          "kv_len": "U[1,%d]" % w.Tkv if w.ragged else (w.kv_len or w.Tkv),
          "nan_padding": w.nan_pad, "sigma": w.sigma,
+         "kv_layout": ("paged [num_pages, Hkv, %d, d], shuffled pages" % page_size) if page_size else "contiguous",
          "l2": "flushed between timed steps (256 MB write)"}
     return c
+
+
+def paged_inputs(w: Workload, inp, page_size: int):
+    """The workload's K/V as a paged cache (storage only; same logical keys)."""
+    lens = inp.kv_lens if inp.kv_lens is not None else torch.full((w.B,), w.Tkv, dtype=torch.int32)
+    kc, vc, table = paginate(inp.k, inp.v, lens, page_size, seed=w.seed)
+    return kc, vc, table, lens
 
 
 def run_ours(args, w, ws, rank, local):
@@ -288,9 +296,17 @@ def run_ours(args, w, ws, rank, local):
     stream = torch.cuda.current_stream(dev)
     nbytes, nflops = workload_work(w, inp.kv_lens)
     unit, bound = metric_unit(w)
+    if args.page_size:
+        kc, vc, table, lens = (t.to(dev) for t in paged_inputs(w, inp, args.page_size))
+        del k, v
 
     def step():
-        binding.gqa_attention_fwd(q, k, v, kv, sink, out, lse, scale=inp.scale, causal=inp.causal, stream=stream)
+        if args.page_size:
+            binding.gqa_attention_fwd_paged(q, kc, vc, table, lens, sink, out, lse, scale=inp.scale,
+                                            causal=inp.causal, stream=stream)
+        else:
+            binding.gqa_attention_fwd(q, k, v, kv, sink, out, lse, scale=inp.scale, causal=inp.causal,
+                                      stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -339,7 +355,7 @@ def run_ours(args, w, ws, rank, local):
     else:
         achieved = nflops / (main_avg / 1e3) / 1e12
         peak = float(peaks["bf16_tflops"])
-    traffic = traffic_for(w)
+    traffic = None if args.page_size else traffic_for(w)
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": traffic, "peak_source": peak_src + (" (burst)" if bound == "tensor" else ""),
                 "kernel": main_kernel_name(w), "kernel_ms": main_avg, "launches_per_step": launches_per_call(w),
@@ -359,7 +375,7 @@ def run_ours(args, w, ws, rank, local):
         line = {
             "metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(w),
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(w, args.page_size),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": len(main_ms) * launches_per_call(w),
             "clocks": clocks,
         }
@@ -368,17 +384,24 @@ def run_ours(args, w, ws, rank, local):
 
 def run_e2e(args, w, inp, dev, stream, nbytes, nflops, ws):
     from gqa_attention_forward_flash_b200 import binding
-    hq, hk, hv = inp.q.pin_memory(), inp.k.pin_memory(), inp.v.pin_memory()
-    hkv = None if inp.kv_lens is None else inp.kv_lens.pin_memory()
+    paged = bool(getattr(args, "page_size", 0))
+    if paged:
+        kc, vc, table, lens = paged_inputs(w, inp, args.page_size)
+        hq, hk, hv, hkv, htab = (t.pin_memory() for t in (inp.q, kc, vc, lens, table))
+    else:
+        hq, hk, hv = inp.q.pin_memory(), inp.k.pin_memory(), inp.v.pin_memory()
+        hkv = None if inp.kv_lens is None else inp.kv_lens.pin_memory()
+        htab = None
     hs = None if inp.sink is None else inp.sink.pin_memory()
     dq, dk, dv = torch.empty_like(hq, device=dev), torch.empty_like(hk, device=dev), torch.empty_like(hv, device=dev)
     dkv = None if hkv is None else torch.empty_like(hkv, device=dev)
+    dtab = None if htab is None else torch.empty_like(htab, device=dev)
     ds = None if hs is None else torch.empty_like(hs, device=dev)
     dout = torch.empty_like(dq)
     dlse = torch.empty((w.B, w.Hq, w.Tq), dtype=torch.float32, device=dev)
     hout = torch.empty_like(hq).pin_memory()
     hlse = torch.empty((w.B, w.Hq, w.Tq), dtype=torch.float32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hkv, hs) if t is not None)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hkv, hs, htab) if t is not None)
     d2h = hout.numel() * hout.element_size() + hlse.numel() * 4
 
     def e2e_step():
@@ -387,10 +410,16 @@ def run_e2e(args, w, inp, dev, stream, nbytes, nflops, ws):
         dv.copy_(hv, non_blocking=True)
         if dkv is not None:
             dkv.copy_(hkv, non_blocking=True)
+        if dtab is not None:
+            dtab.copy_(htab, non_blocking=True)
         if ds is not None:
             ds.copy_(hs, non_blocking=True)
-        binding.gqa_attention_fwd(dq, dk, dv, dkv, ds, dout, dlse, scale=inp.scale, causal=inp.causal,
-                                  stream=stream)
+        if paged:
+            binding.gqa_attention_fwd_paged(dq, dk, dv, dtab, dkv, ds, dout, dlse, scale=inp.scale,
+                                            causal=inp.causal, stream=stream)
+        else:
+            binding.gqa_attention_fwd(dq, dk, dv, dkv, ds, dout, dlse, scale=inp.scale, causal=inp.causal,
+                                      stream=stream)
         hout.copy_(dout, non_blocking=True)
         hlse.copy_(dlse, non_blocking=True)
 
@@ -464,6 +493,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-step-seconds", type=float, default=3.0)
     ap.add_argument("--burn-seconds", type=float, default=1.5)
+    ap.add_argument("--page-size", type=int, default=0,
+                    help="read K/V through gqa_attention_fwd_paged from a cache of pages of this many tokens "
+                         "(0: contiguous K/V through gqa_attention_fwd)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libgqa_attn.so")
 STATUS = {
     0: "GQA_OK", -1: "GQA_ERR_NULL", -2: "GQA_ERR_SHAPE", -3: "GQA_ERR_ALIGN", -4: "GQA_ERR_SPLITS",
     -5: "GQA_ERR_CUDA", -6: "GQA_ERR_TIMEOUT", -7: "GQA_ERR_UNSUPPORTED", -8: "GQA_ERR_KVLEN",
-    -9: "GQA_ERR_SCRATCH",
+    -9: "GQA_ERR_SCRATCH", -10: "GQA_ERR_PAGE",
 }
 MAX_SPLITS = 256
 
@@ -27,6 +27,7 @@ _P, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 SIGNATURES = {
     "gqa_attention_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "gqa_attention_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "gqa_attention_fwd_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "gqa_attention_fwd_partial": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P, _P]),
     "gqa_splitkv_combine": (_I, [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
     "gqa_get_device_error": (_I, [_P]),
@@ -102,6 +103,34 @@ def gqa_attention_fwd(q, k, v, kv_lens=None, sink=None, out=None, lse=None, scal
     rc = load().gqa_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_lens), _ptr(sink), _ptr(out), _ptr(lse),
                                   B, Hq, Hkv, Tq, Tkv, d, float(scale), int(bool(causal)), _stream(stream))
     _check("gqa_attention_fwd", rc)
+    return out, lse
+
+
+def gqa_attention_fwd_paged(q, k_cache, v_cache, page_table, kv_lens, sink=None, out=None, lse=None, scale=None,
+                            causal=False, stream=None):
+    """The forward over a paged K/V cache.  q [B,Hq,Tq,d] bf16; k_cache/v_cache
+    [num_pages, Hkv, page_size, d] bf16; page_table int32 [B, max_pages];
+    kv_lens int32 [B] (required); sink fp32 [Hq] or None.  Returns (out, lse)."""
+    _need(q, torch.bfloat16, "q", 4)
+    _need(k_cache, torch.bfloat16, "k_cache", 4)
+    _need(v_cache, torch.bfloat16, "v_cache", 4)
+    _need(page_table, torch.int32, "page_table", 2)
+    _need(kv_lens, torch.int32, "kv_lens", 1)
+    B, Hq, Tq, d = q.shape
+    num_pages, Hkv, page_size, _ = k_cache.shape
+    max_pages = page_table.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=q.device)
+    if sink is not None:
+        _need(sink, torch.float32, "sink", 1)
+    if scale is None:
+        scale = d ** -0.5
+    rc = load().gqa_attention_fwd_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(page_table), _ptr(kv_lens),
+                                        _ptr(sink), _ptr(out), _ptr(lse), B, Hq, Hkv, Tq, num_pages, page_size,
+                                        max_pages, d, float(scale), int(bool(causal)), _stream(stream))
+    _check("gqa_attention_fwd_paged", rc)
     return out, lse
 
 

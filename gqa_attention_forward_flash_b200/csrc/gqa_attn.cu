@@ -200,18 +200,25 @@ int launch_fwd(const Params& p0, const void* q, const void* k, const void* v, in
     // padding rows (query rows past the group, or key rows past kv_len, which the
     // kernel zeroes in V and masks in S)
     const uint64_t qrows = static_cast<uint64_t>(p.B) * p.Hq * p.Tq;
-    const uint64_t kvrows = static_cast<uint64_t>(p.B) * p.Hkv * p.Tkv;
+    // paged K/V: the caches viewed as [num_pages*Hkv*page_size, d], one box per page piece
+    const bool paged = p.page_size > 0;
+    const uint64_t kvrows = paged ? static_cast<uint64_t>(p.num_pages) * p.Hkv * p.page_size
+                                  : static_cast<uint64_t>(p.B) * p.Hkv * p.Tkv;
+    const uint64_t kvcols = static_cast<uint64_t>(C::D);
     // few packed rows (decode): spread them over the four TMEM lane quadrants so
     // that every SM sub-partition takes a share of the softmax
     p.spread = (p.QT == 1 && p.R <= 96) ? 1 : 0;
     p.rq = (p.R + 3) / 4;
     p.q_box_rows = p.spread ? p.rq : (qrows < static_cast<uint64_t>(BM) ? static_cast<int>(qrows) : BM);
-    p.kv_box_rows = kvrows < static_cast<uint64_t>(C::BN) ? static_cast<int>(kvrows) : C::BN;
+    if (paged)
+        p.kv_box_rows = p.page_size < C::BN ? p.page_size : C::BN;
+    else
+        p.kv_box_rows = kvrows < static_cast<uint64_t>(C::BN) ? static_cast<int>(kvrows) : C::BN;
     int rc = make_tmap(&tq, q, qrows, C::D, p.q_box_rows);
     if (rc) return rc;
-    rc = make_tmap(&tk, k, kvrows, C::D, p.kv_box_rows);
+    rc = make_tmap(&tk, k, kvrows, kvcols, p.kv_box_rows);
     if (rc) return rc;
-    rc = make_tmap(&tv, v, kvrows, C::D, p.kv_box_rows);
+    rc = make_tmap(&tv, v, kvrows, kvcols, p.kv_box_rows);
     if (rc) return rc;
     if (ev_before && cudaEventRecord(ev_before, stream) != cudaSuccess) return GQA_ERR_CUDA;
     if constexpr (TWO_LANE)
@@ -277,32 +284,19 @@ int ensure_scratch(DeviceState& s, size_t bytes) {
     return GQA_OK;
 }
 
-}  // namespace
-}  // namespace gqa
-
-using namespace gqa;
-
-extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, const int32_t* kv_lens,
-                                 const float* sink, void* out, float* lse, int B, int Hq, int Hkv, int Tq,
-                                 int Tkv, int d, float scale, int causal, gqa_stream_t stream) {
-    int rc = check_common(q, k, v, B, Hq, Hkv, Tq, Tkv, d, scale);
-    if (rc) return rc;
-    if (B == 0 || Tq == 0) return GQA_OK;
-    if (!out) return GQA_ERR_NULL;
-    if (!aligned16(out) || (lse && !aligned16(lse))) return GQA_ERR_ALIGN;
-    std::lock_guard<std::mutex> lk(g_mu);
-    DeviceState* s = nullptr;
-    rc = get_state(&s);
-    if (rc) return rc;
-    if (s->cc_major != 10) return GQA_ERR_UNSUPPORTED;
-    Params p;
-    fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale, causal, kv_lens, sink, out, lse, 0, timeout_cycles(*s));
+// The stream-K forward shared by the contiguous and the paged entry points:
+// plan, scratch, launch (and the combine launch for head dims 256 / 512).
+int run_streamk(Params& p, const void* q, const void* k, const void* v, DeviceState& sr, gqa_stream_t stream) {
+    DeviceState* s = &sr;
+    const int d = p.d, Tkv = p.Tkv;
+    const bool has_lens = p.kv_lens != nullptr;
+    int rc = GQA_OK;
     choose_geometry(p);
     // grid: one CTA per SM (NC groups of DSPLIT CTAs); with host-known lengths never
     // more groups than tiles
     const int ds = dsplit_for(d);
     int NC = (s->sm_count < kMaxCtas ? s->sm_count : kMaxCtas) / ds;
-    if (!kv_lens) {
+    if (!has_lens) {
         long long tot = 0;
         for (int qw = 0; qw < p.QW; ++qw) tot += qtile_ntiles(p, qw, Tkv);
         tot *= p.U;
@@ -341,6 +335,58 @@ extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, co
         if (ev && cudaEventRecord(ev[1], st) != cudaSuccess) return GQA_ERR_CUDA;
     }
     return GQA_OK;
+}
+
+}  // namespace
+}  // namespace gqa
+
+using namespace gqa;
+
+extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, const int32_t* kv_lens,
+                                 const float* sink, void* out, float* lse, int B, int Hq, int Hkv, int Tq,
+                                 int Tkv, int d, float scale, int causal, gqa_stream_t stream) {
+    int rc = check_common(q, k, v, B, Hq, Hkv, Tq, Tkv, d, scale);
+    if (rc) return rc;
+    if (B == 0 || Tq == 0) return GQA_OK;
+    if (!out) return GQA_ERR_NULL;
+    if (!aligned16(out) || (lse && !aligned16(lse))) return GQA_ERR_ALIGN;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState* s = nullptr;
+    rc = get_state(&s);
+    if (rc) return rc;
+    if (s->cc_major != 10) return GQA_ERR_UNSUPPORTED;
+    Params p;
+    fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale, causal, kv_lens, sink, out, lse, 0, timeout_cycles(*s));
+    return run_streamk(p, q, k, v, *s, stream);
+}
+
+extern "C" int gqa_attention_fwd_paged(const void* q, const void* k_cache, const void* v_cache,
+                                       const int32_t* page_table, const int32_t* kv_lens, const float* sink, void* out,
+                                       float* lse, int B, int Hq, int Hkv, int Tq, int num_pages, int page_size,
+                                       int max_pages, int d, float scale, int causal, gqa_stream_t stream) {
+    if (page_size < 8 || page_size > 1024 || (page_size & (page_size - 1)) != 0) return GQA_ERR_SHAPE;
+    if (num_pages < 1 || max_pages < 1) return GQA_ERR_SHAPE;
+    if (static_cast<long long>(max_pages) * page_size >= (1ll << 30)) return GQA_ERR_SHAPE;
+    if (static_cast<long long>(num_pages) * (Hkv > 0 ? Hkv : 1) * page_size + 256 >= (1ll << 31)) return GQA_ERR_SHAPE;
+    const int Tkv = max_pages * page_size;  // a sequence's capacity
+    int rc = check_common(q, k_cache, v_cache, B, Hq, Hkv, Tq, Tkv, d, scale);
+    if (rc) return rc;
+    if (d != 64 && d != 128) return GQA_ERR_UNSUPPORTED;
+    if (B == 0 || Tq == 0) return GQA_OK;
+    if (!out || !page_table || !kv_lens) return GQA_ERR_NULL;
+    if (!aligned16(out) || (lse && !aligned16(lse))) return GQA_ERR_ALIGN;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState* s = nullptr;
+    rc = get_state(&s);
+    if (rc) return rc;
+    if (s->cc_major != 10) return GQA_ERR_UNSUPPORTED;
+    Params p;
+    fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale, causal, kv_lens, sink, out, lse, 0, timeout_cycles(*s));
+    p.page_table = page_table;
+    p.page_size = page_size;
+    p.max_pages = max_pages;
+    p.num_pages = num_pages;
+    return run_streamk(p, q, k_cache, v_cache, *s, stream);
 }
 
 extern "C" int gqa_attention_fwd_partial(const void* q, const void* k, const void* v, const int32_t* kv_lens,
@@ -457,6 +503,7 @@ extern "C" const char* gqa_status_string(int status) {
         case GQA_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
         case GQA_ERR_UNSUPPORTED: return "unsupported head dim or GPU";
         case GQA_ERR_KVLEN: return "a kv_lens value was outside [0, Tkv] and was clamped";
+        case GQA_ERR_PAGE: return "a page id was outside [0, num_pages); page 0 was read instead";
         case GQA_ERR_SCRATCH: return "the problem needs more scratch than the fixed allocation-free array holds";
         default: return "unknown status";
     }

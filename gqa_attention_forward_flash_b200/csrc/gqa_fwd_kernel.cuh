@@ -57,6 +57,7 @@ constexpr int kMaxCombinePieces = 512;  // CTA groups of a split (the grid is at
 // device error codes (same values as gqa_status)
 constexpr int DEV_ERR_TIMEOUT = -6;
 constexpr int DEV_ERR_KVLEN = -8;
+constexpr int DEV_ERR_PAGE = -10;
 
 // A split row-block (one DSPLIT part of its O columns) whose pieces are all
 // written: the stream-K combine kernel merges it.
@@ -95,6 +96,12 @@ struct Params {
     int kv_box_rows;      // rows of one K/V TMA box: min(BN, B*Hkv*Tkv)
     CJob* cjobs;          // single-lane kernel, mode 0: [W*DSPLIT] row-blocks for the combine kernel
     int* cjob_count;      // [2]: jobs listed, combine blocks done (zero between calls)
+    // paged K/V (two-lane kernel): caches [num_pages, Hkv, page_size, d], page_table
+    // [B, max_pages] (logical page -> physical page); page_size 0 = contiguous K/V
+    const int* page_table;
+    int page_size;
+    int max_pages;
+    int num_pages;
 };
 
 // ------------------------------------------------------------------ schedule

@@ -117,3 +117,33 @@ def make_inputs(w: Workload, seed: int | None = None) -> Inputs:
     sink = torch.randn((w.Hq,), generator=g, dtype=torch.float32) if w.sink else None
     return Inputs(q=q, k=k, v=v, kv_lens=kv_lens, sink=sink, scale=w.scale, causal=w.causal)
 
+
+
+def paginate(k, v, kv_lens, page_size: int, seed: int, spare_pages: int = 3):
+    """Store contiguous K/V [B, Hkv, Tkv, d] as a paged cache: pages of page_size
+    tokens laid out [num_pages, Hkv, page_size, d], each sequence's pages at
+    shuffled physical positions among spare NaN-filled pages, and a page table
+    int32 [B, max_pages] whose entries past a sequence's pages are -1 (never read).
+    Storage layout only: the keys and values of every logical position are those
+    of the contiguous tensors.  Returns (k_cache, v_cache, page_table)."""
+    B, Hkv, Tkv, d = k.shape
+    max_pages = (Tkv + page_size - 1) // page_size
+    lens = [int(x) for x in kv_lens.tolist()]
+    used = [(len_ + page_size - 1) // page_size for len_ in lens]
+    num_pages = sum(used) + spare_pages
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    order = torch.randperm(num_pages, generator=g).tolist()
+    k_cache = torch.full((num_pages, Hkv, page_size, d), float("nan"), dtype=k.dtype)
+    v_cache = torch.full((num_pages, Hkv, page_size, d), float("nan"), dtype=v.dtype)
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    nxt = 0
+    for b in range(B):
+        for j in range(used[b]):
+            phys = order[nxt]
+            nxt += 1
+            table[b, j] = phys
+            lo, hi = j * page_size, min((j + 1) * page_size, Tkv)
+            k_cache[phys, :, : hi - lo] = k[b, :, lo:hi, :]
+            v_cache[phys, :, : hi - lo] = v[b, :, lo:hi, :]
+    return k_cache, v_cache, table

@@ -75,7 +75,8 @@ typedef enum {
     GQA_ERR_TIMEOUT = -6,     /* a bounded wait inside a kernel ran out (device-reported) */
     GQA_ERR_UNSUPPORTED = -7, /* head dim not in {64,128,256,512}, or the GPU is not sm_100 */
     GQA_ERR_KVLEN = -8,       /* a kv_lens value was outside [0, Tkv] (device-reported, clamped) */
-    GQA_ERR_SCRATCH = -9      /* gqa_attention_fwd_noalloc: the problem exceeds its fixed scratch */
+    GQA_ERR_SCRATCH = -9,     /* gqa_attention_fwd_noalloc: the problem exceeds its fixed scratch */
+    GQA_ERR_PAGE = -10        /* gqa_attention_fwd_paged: a page id outside [0, num_pages) (device-reported) */
 } gqa_status;
 
 #define GQA_MAX_SPLITS 256
@@ -116,6 +117,31 @@ int gqa_attention_fwd_partial(const void *q, const void *k, const void *v, const
 int gqa_splitkv_combine(const float *o_part, const float *lse_part, int num_splits,
                         const float *sink, void *out, float *lse, int B, int Hq, int Tq, int d,
                         gqa_stream_t stream);
+
+/*
+ * gqa_attention_fwd over a paged K/V cache (AstrAI commit log, attention
+ * commits: a KV-source policy selecting contiguous or paged K/V, page-table and
+ * cache-location indices stored as int32, the paged decode address path).  The
+ * pages give no cache layout; this one is the common one:
+ *   k_cache, v_cache: bf16 [num_pages, Hkv, page_size, d], contiguous, caller-owned
+ *                     (head-major pages: one (page, KV head) block is contiguous, so
+ *                     a key tile of one head is read as whole pages);
+ *   page_table:       int32 [B, max_pages] (device): logical page j of batch b is
+ *                     physical page page_table[b * max_pages + j]; entries past
+ *                     ceil(kv_lens[b] / page_size) are never read;
+ *   kv_lens:          int32 [B] (device, required): logical lengths, each in
+ *                     [0, max_pages * page_size] (else clamped, GQA_ERR_KVLEN).
+ * Q, out and lse are dense as in gqa_attention_fwd; so are sink, scale, causal
+ * (bottom-right against kv_lens[b]).  page_size is a power of two in [8, 1024];
+ * d in {64, 128} (GQA_ERR_UNSUPPORTED otherwise).  A page id outside
+ * [0, num_pages) makes the kernel read page 0 instead and report GQA_ERR_PAGE
+ * through gqa_get_device_error.  Same scratch and error behaviour as
+ * gqa_attention_fwd.
+ */
+int gqa_attention_fwd_paged(const void *q, const void *k_cache, const void *v_cache, const int32_t *page_table,
+                            const int32_t *kv_lens, const float *sink, void *out, float *lse, int B, int Hq,
+                            int Hkv, int Tq, int num_pages, int page_size, int max_pages, int d, float scale,
+                            int causal, gqa_stream_t stream);
 
 /*
  * gqa_attention_fwd without any device allocation.  The pages have no

@@ -99,3 +99,19 @@ def test_valid_call_without_a_gpu_fails_loudly(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert fwd(lib) == -5  # GQA_ERR_CUDA: no silent CPU path
+
+
+def paged(lib, page_size=64, d=64, table=16, lens=16, num_pages=8, max_pages=4):
+    return lib.gqa_attention_fwd_paged(P(16), P(16), P(16), P(table), P(lens), None, P(16), P(16), 1, 4, 1, 4,
+                                       num_pages, page_size, max_pages, d, 0.125, 0, None)
+
+
+def test_paged_entry_rejects_bad_arguments_on_the_host(lib):
+    assert paged(lib, page_size=48) == -2      # not a power of two
+    assert paged(lib, page_size=4) == -2       # below 8
+    assert paged(lib, page_size=2048) == -2    # above 1024
+    assert paged(lib, num_pages=0) == -2
+    assert paged(lib, max_pages=0) == -2
+    assert paged(lib, d=256) == -7             # only head dims 64 and 128
+    assert paged(lib, table=None) == -1        # page table required
+    assert paged(lib, lens=None) == -1         # kv_lens required
