@@ -16,7 +16,7 @@
 #include <mutex>
 
 #include "gqa_attn.h"
-#include "gqa_fwd2_kernel.cuh"
+#include "gqa_dec_kernel.cuh"
 
 namespace gqa {
 namespace {
@@ -146,6 +146,19 @@ using C2_64_SK = Fwd2Cfg<64, 4, 4, 1>;
 using C2_64_DQ = Fwd2Cfg<64, 4, 4, 2>;
 using C2_128_SK = Fwd2Cfg<128, 3, 3, 1>;
 using C2_128_DQ = Fwd2Cfg<128, 3, 2, 2>;
+// the same four over a paged K/V cache (a separate instantiation keeps the
+// page-table producer out of the contiguous kernels)
+using C2_64_SK_P = Fwd2Cfg<64, 4, 4, 1, true>;
+using C2_64_DQ_P = Fwd2Cfg<64, 4, 4, 2, true>;
+using C2_128_SK_P = Fwd2Cfg<128, 3, 3, 1, true>;
+using C2_128_DQ_P = Fwd2Cfg<128, 3, 2, 2, true>;
+// Few packed rows (decode) at head dim 128: the swap-AB kernel, reading 8 or 16
+// rows of its transposed tiles
+using CDec8 = DecCfg<8>;
+using CDec16 = DecCfg<16>;
+using CDec8_P = DecCfg<8, true>;
+using CDec16_P = DecCfg<16, true>;
+bool uses_decode_kernel(const Params& p) { return p.d == 128 && p.mode == 0 && p.R <= DEC_NQ; }
 using Cfg256 = FwdCfg<256, 64, 3, 2, 1>;
 // Head dim 512: O (128 x 512 fp32) fills a whole TMEM, so O's columns are split
 // over a pair of CTAs (DSPLIT = 2) that each compute the full S.
@@ -179,7 +192,11 @@ void choose_geometry(Params& p) {
     p.W = static_cast<long long>(p.U) * p.QW;
 }
 
-template <class C, bool TWO_LANE>
+// Kernel families: the single-lane kernel (head dims 256, 512), the two-lane
+// kernel (64, 128) and the swap-AB decode kernel (128, at most 16 packed rows).
+enum KernelKind { kSingleLane = 0, kTwoLane = 1, kDecode = 2 };
+
+template <class C, int KIND>
 int launch_fwd(const Params& p0, const void* q, const void* k, const void* v, int grid, cudaStream_t stream,
                cudaEvent_t ev_before, cudaEvent_t ev_after) {
     static bool attr_done[kMaxDevices] = {};
@@ -187,8 +204,10 @@ int launch_fwd(const Params& p0, const void* q, const void* k, const void* v, in
     if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
     if (!attr_done[dev]) {
         cudaError_t e;
-        if constexpr (TWO_LANE)
+        if constexpr (KIND == kTwoLane)
             e = cudaFuncSetAttribute(gqa_fwd2_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        else if constexpr (KIND == kDecode)
+            e = cudaFuncSetAttribute(gqa_dec_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         else
             e = cudaFuncSetAttribute(gqa_fwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return GQA_ERR_CUDA;
@@ -207,9 +226,12 @@ int launch_fwd(const Params& p0, const void* q, const void* k, const void* v, in
     const uint64_t kvcols = static_cast<uint64_t>(C::D);
     // few packed rows (decode): spread them over the four TMEM lane quadrants so
     // that every SM sub-partition takes a share of the softmax
-    p.spread = (p.QT == 1 && p.R <= 96) ? 1 : 0;
+    p.spread = (KIND != kDecode && p.QT == 1 && p.R <= 96) ? 1 : 0;
     p.rq = (p.R + 3) / 4;
-    p.q_box_rows = p.spread ? p.rq : (qrows < static_cast<uint64_t>(BM) ? static_cast<int>(qrows) : BM);
+    if constexpr (KIND == kDecode)  // the 16-row Q tile of the transposed MMAs
+        p.q_box_rows = qrows < static_cast<uint64_t>(DEC_NQ) ? static_cast<int>(qrows) : DEC_NQ;
+    else
+        p.q_box_rows = p.spread ? p.rq : (qrows < static_cast<uint64_t>(BM) ? static_cast<int>(qrows) : BM);
     if (paged)
         p.kv_box_rows = p.page_size < C::BN ? p.page_size : C::BN;
     else
@@ -221,8 +243,10 @@ int launch_fwd(const Params& p0, const void* q, const void* k, const void* v, in
     rc = make_tmap(&tv, v, kvrows, kvcols, p.kv_box_rows);
     if (rc) return rc;
     if (ev_before && cudaEventRecord(ev_before, stream) != cudaSuccess) return GQA_ERR_CUDA;
-    if constexpr (TWO_LANE)
+    if constexpr (KIND == kTwoLane)
         gqa_fwd2_kernel<C><<<grid, NUM_THREADS2, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    else if constexpr (KIND == kDecode)
+        gqa_dec_kernel<C><<<grid, NUM_THREADS_DEC, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     else
         gqa_fwd_kernel<C><<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
@@ -234,13 +258,26 @@ int dispatch_fwd(const Params& p, const void* q, const void* k, const void* v, i
                  cudaEvent_t e0 = nullptr, cudaEvent_t e1 = nullptr) {
     switch (p.d) {
         case 64:
-            return p.RBQ == 1 ? launch_fwd<C2_64_SK, true>(p, q, k, v, grid, stream, e0, e1)
-                              : launch_fwd<C2_64_DQ, true>(p, q, k, v, grid, stream, e0, e1);
+            if (p.page_size > 0)
+                return p.RBQ == 1 ? launch_fwd<C2_64_SK_P, kTwoLane>(p, q, k, v, grid, stream, e0, e1)
+                                  : launch_fwd<C2_64_DQ_P, kTwoLane>(p, q, k, v, grid, stream, e0, e1);
+            return p.RBQ == 1 ? launch_fwd<C2_64_SK, kTwoLane>(p, q, k, v, grid, stream, e0, e1)
+                              : launch_fwd<C2_64_DQ, kTwoLane>(p, q, k, v, grid, stream, e0, e1);
         case 128:
-            return p.RBQ == 1 ? launch_fwd<C2_128_SK, true>(p, q, k, v, grid, stream, e0, e1)
-                              : launch_fwd<C2_128_DQ, true>(p, q, k, v, grid, stream, e0, e1);
-        case 256: return launch_fwd<Cfg256, false>(p, q, k, v, grid, stream, e0, e1);
-        case 512: return launch_fwd<Cfg512, false>(p, q, k, v, grid, stream, e0, e1);
+            if (uses_decode_kernel(p)) {
+                if (p.page_size > 0)
+                    return p.R <= 8 ? launch_fwd<CDec8_P, kDecode>(p, q, k, v, grid, stream, e0, e1)
+                                    : launch_fwd<CDec16_P, kDecode>(p, q, k, v, grid, stream, e0, e1);
+                return p.R <= 8 ? launch_fwd<CDec8, kDecode>(p, q, k, v, grid, stream, e0, e1)
+                                : launch_fwd<CDec16, kDecode>(p, q, k, v, grid, stream, e0, e1);
+            }
+            if (p.page_size > 0)
+                return p.RBQ == 1 ? launch_fwd<C2_128_SK_P, kTwoLane>(p, q, k, v, grid, stream, e0, e1)
+                                  : launch_fwd<C2_128_DQ_P, kTwoLane>(p, q, k, v, grid, stream, e0, e1);
+            return p.RBQ == 1 ? launch_fwd<C2_128_SK, kTwoLane>(p, q, k, v, grid, stream, e0, e1)
+                              : launch_fwd<C2_128_DQ, kTwoLane>(p, q, k, v, grid, stream, e0, e1);
+        case 256: return launch_fwd<Cfg256, kSingleLane>(p, q, k, v, grid, stream, e0, e1);
+        case 512: return launch_fwd<Cfg512, kSingleLane>(p, q, k, v, grid, stream, e0, e1);
         default: return GQA_ERR_UNSUPPORTED;
     }
 }

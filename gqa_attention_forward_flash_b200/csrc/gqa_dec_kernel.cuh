@@ -1,0 +1,691 @@
+// gqa_dec_kernel.cuh -- sm_100a GQA forward for few packed query rows (decode):
+// at most 16 packed rows R = G*Tq per (batch, KV head), head dim 128.
+//
+// With so few query rows a 128-row MMA tile would be almost all padding, and so
+// would the softmax work of one thread per query row.  Here both contractions are
+// computed transposed ("swap AB"), so the 128 keys of a tile are the MMA's M
+// dimension and the query rows its N = 16:
+//
+//   S' = K Q^T   [128 keys x 16 rows]   TMEM lanes = keys
+//   O' = V^T P'  [128 dims x 16 rows]   TMEM lanes = head dims
+//
+// One softmax thread per key holds at most 16 scores of a tile; the row maxima
+// are reduced over the 128 keys once per tile (warp butterfly, then the four
+// warps through shared memory); each thread keeps partial row sums of its own
+// keys, reduced once per segment.  P'^T (bf16, 16 rows x 128 keys, K-major,
+// 128-byte swizzle) goes to shared memory as the B operand of the second MMA;
+// V's shared-memory tile serves as the MN-major A operand V^T unchanged.
+//
+//   TMEM columns  [0,16) S'0   [16,32) S'1   [32,48) O'
+//
+// MMA order (one thread): S'(g), PV'(g-1), S'(g+1), PV'(g), ...  S' is double
+// buffered; P' is double buffered; the softmax of tile g overlaps PV'(g-1).
+// Warps: 0 Q/K producer (and the stream-K plan), 1 V producer, 2 TMEM owner +
+// MMA issuer, 3 split-segment ticket taker, 4-7 softmax (warp 4+q reads TMEM
+// lane quadrant q).  The stream-K work split, the split partial slots and the
+// last-arriver merge are those of the two-lane kernel (gqa_fwd2_kernel.cuh).
+#pragma once
+#include "gqa_fwd2_kernel.cuh"
+
+namespace gqa {
+
+constexpr int NUM_THREADS_DEC = 256;
+constexpr int NSOFT_DEC = 128;
+constexpr int DEC_NQ = 16;  // N of both MMAs: packed query rows held (padded)
+
+template <int NR_, bool PAGED_ = false>
+struct DecCfg {
+    static constexpr int D = 128, BN = 128, STK = 3, STV = 3, QBUF = 2;
+    static constexpr int NR = NR_;  // query rows the softmax reads (8 or 16)
+    static_assert(NR == 8 || NR == 16, "rows");
+    static constexpr bool PAGED = PAGED_;
+    static constexpr int NBOX = D / 64;
+    static constexpr int KV_BOX = BN * 128;             // one 64-column box of a K/V tile
+    static constexpr int KV_BYTES = NBOX * KV_BOX;
+    static constexpr int Q_BOX = DEC_NQ * 128;          // one 64-column box of the 16-row Q tile
+    static constexpr int Q_BYTES = NBOX * Q_BOX;
+    static constexpr int P_BOX = DEC_NQ * 128;          // one 64-key box of P'^T
+    static constexpr int P_BYTES = (BN / 64) * P_BOX;
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = OFF_K + STK * KV_BYTES;
+    static constexpr int OFF_Q = OFF_V + STV * KV_BYTES;
+    static constexpr int OFF_P = OFF_Q + QBUF * Q_BYTES;
+    static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+    static constexpr int B_QFULL = 0;                   // [QBUF]
+    static constexpr int B_QEMPTY = B_QFULL + QBUF;     // [QBUF]
+    static constexpr int B_KFULL = B_QEMPTY + QBUF;
+    static constexpr int B_KEMPTY = B_KFULL + STK;
+    static constexpr int B_VFULL = B_KEMPTY + STK;
+    static constexpr int B_VEMPTY = B_VFULL + STV;
+    static constexpr int B_SFULL = B_VEMPTY + STV;      // [2] S' buffer written
+    static constexpr int B_PFULL = B_SFULL + 2;         // [2] P' buffer written (one arrival per softmax warp)
+    static constexpr int B_PVDONE = B_PFULL + 2;        // [2] PV' that read P' buffer b completed
+    static constexpr int B_OFREE = B_PVDONE + 2;        // segment epilogue has read O'
+    static constexpr int B_RED = B_OFREE + 1;           // softmax warps: per-tile row reductions
+    static constexpr int B_XSYNC = B_RED + 1;           // softmax warps: epilogue / merge steps
+    static constexpr int B_FINAL = B_XSYNC + 1;
+    static constexpr int B_MJOB = B_FINAL + 1;          // [2] partial rows of split segment j written
+    static constexpr int B_MTICK = B_MJOB + 2;          // [2] ticket of split segment j taken
+    static constexpr int NBAR = B_MTICK + 2;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int MISC_BYTES = 1536;
+    static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES;
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+    static constexpr uint32_t TM_COLS = 64;
+    static constexpr uint32_t TM_S = 0;   // + 16 * buffer
+    static constexpr uint32_t TM_O = 32;
+    static constexpr uint32_t IDESC_S = ptx::umma_idesc_bf16_f32(BN, DEC_NQ, false, false);
+    static constexpr uint32_t IDESC_PV = ptx::umma_idesc_bf16_f32(D, DEC_NQ, true, false);
+};
+
+struct DecMisc {
+    uint32_t tmem_base;       // the first four fields match Misc (bounded waits read abort)
+    volatile int abort;
+    volatile int merge_flag;
+    int pad;
+    SpanStart span;
+    float red[2][DEC_NQ][4];  // per-tile row reductions: [phase][row][softmax warp]
+    float mlse[DEC_NQ];       // merged lse per packed row (in-kernel merge)
+    int nmerge;
+    int mslot[kMaxMergeSlots];
+    Seg jobs[2];
+    int ticket[2];
+};
+
+// Reduce NR per-thread values over the 32 lanes of a warp, one row per lane group:
+// returns the reduction of row dec_row_of<NR>(lane).  Each halving step trades the
+// half a lane does not keep with its partner, so 2*NR - 1 shuffles in all.
+template <int NR, bool MAX>
+__device__ __forceinline__ float dec_warp_reduce(const float (&x)[NR], int lane) {
+    float v[NR];
+#pragma unroll
+    for (int i = 0; i < NR; ++i) v[i] = x[i];
+    int bit = 16;
+#pragma unroll
+    for (int step = NR / 2; step >= 1; step /= 2, bit >>= 1) {
+        const bool up = (lane & bit) != 0;
+#pragma unroll
+        for (int i = 0; i < step; ++i) {
+            const float keep = up ? v[i + step] : v[i];
+            const float send = up ? v[i] : v[i + step];
+            const float got = __shfl_xor_sync(0xffffffffu, send, bit);
+            v[i] = MAX ? fmaxf(keep, got) : keep + got;
+        }
+    }
+#pragma unroll
+    for (int b = bit; b >= 1; b >>= 1) {
+        const float got = __shfl_xor_sync(0xffffffffu, v[0], b);
+        v[0] = MAX ? fmaxf(v[0], got) : v[0] + got;
+    }
+    return v[0];
+}
+template <int NR>
+__device__ __forceinline__ int dec_row_of(int lane) {
+    return (NR == 8) ? (((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1))
+                     : (((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1));
+}
+template <int NR>
+__device__ __forceinline__ bool dec_row_writer(int lane) {
+    return (NR == 8) ? (lane & 3) == 0 : (lane & 1) == 0;
+}
+
+template <class C>
+__global__ void __launch_bounds__(NUM_THREADS_DEC, 1)
+gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const Params p) {
+    constexpr int NR = C::NR;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw;
+    const uint32_t sbase = ptx::smem_addr(smem);
+    if (sbase & 1023u) {  // the swizzled tiles need a 1024-aligned window
+        if (threadIdx.x == 0) atomicCAS(p.err, 0, DEV_ERR_TIMEOUT);
+        return;
+    }
+    const uint32_t bar0 = sbase + C::OFF_BAR;
+    auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
+    DecMisc* misc = reinterpret_cast<DecMisc*>(smem + C::OFF_MISC);
+    Misc* wmisc = reinterpret_cast<Misc*>(misc);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int cta = blockIdx.x;
+    const int NC = gridDim.x;
+
+    // ---------------------------------------------------------------- setup
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::QBUF; ++i) {
+            ptx::mbar_init(bar(C::B_QFULL + i), 1);
+            ptx::mbar_init(bar(C::B_QEMPTY + i), 1);
+        }
+        for (int i = 0; i < C::STK; ++i) {
+            ptx::mbar_init(bar(C::B_KFULL + i), 1);
+            ptx::mbar_init(bar(C::B_KEMPTY + i), 1);
+        }
+        for (int i = 0; i < C::STV; ++i) {
+            ptx::mbar_init(bar(C::B_VFULL + i), 1);
+            ptx::mbar_init(bar(C::B_VEMPTY + i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(bar(C::B_SFULL + i), 1);
+            ptx::mbar_init(bar(C::B_PFULL + i), 4);
+            ptx::mbar_init(bar(C::B_PVDONE + i), 1);
+            ptx::mbar_init(bar(C::B_MJOB + i), 1);
+            ptx::mbar_init(bar(C::B_MTICK + i), 1);
+        }
+        ptx::mbar_init(bar(C::B_OFREE), 4);
+        ptx::mbar_init(bar(C::B_RED), 4);
+        ptx::mbar_init(bar(C::B_XSYNC), 4);
+        ptx::mbar_init(bar(C::B_FINAL), 1);
+        misc->abort = 0;
+        misc->merge_flag = 0;
+        ptx::fence_mbar_init();
+        ptx::tma_prefetch_desc(&tm_q);
+        ptx::tma_prefetch_desc(&tm_k);
+        ptx::tma_prefetch_desc(&tm_v);
+    }
+    if (warp == 2) {
+        ptx::tmem_alloc(ptx::smem_addr(&misc->tmem_base), C::TM_COLS);
+        ptx::tmem_relinquish();
+    }
+    if (warp == 0) plan_span(p, cta, NC, &misc->span);
+    if (warp >= 4) {
+        // P' rows past NR are never written by the softmax: keep them zero
+        uint4* pz = reinterpret_cast<uint4*>(smem + C::OFF_P);
+        for (int i = threadIdx.x - 128; i < 2 * C::P_BYTES / 16; i += NSOFT_DEC) pz[i] = make_uint4(0, 0, 0, 0);
+        ptx::fence_proxy_async_smem();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = misc->tmem_base;
+
+    if (warp < 4) {
+        // ------------------------------------------------------------ Q / K producer
+        if (warp == 0 && lane == 0) {
+            const uint64_t pol_q = ptx::policy_evict_last();
+            const uint64_t pol_kv = ptx::policy_evict_first();
+            SegWalker wk;
+            wk.init(p, misc->span, cta);
+            Seg sg;
+            int seg_i = 0;
+            uint32_t g = 0;
+            bool ok = true;
+            uint32_t k_issued[C::STK], q_issued[C::QBUF];
+            for (int i = 0; i < C::STK; ++i) k_issued[i] = 0;
+            for (int i = 0; i < C::QBUF; ++i) q_issued[i] = 0;
+            while (ok && wk.next(p, sg)) {
+                if (sg.t1 <= sg.t0) continue;
+                const RB rb = rb_of(p, sg.w);
+                const int qb = seg_i % C::QBUF;
+                ok = wait_bar(bar(C::B_QEMPTY + qb), ((seg_i / C::QBUF) & 1) ^ 1, wmisc, p);
+                if (!ok) break;
+                ptx::mbar_arrive_expect_tx(bar(C::B_QFULL + qb), C::NBOX * p.q_box_rows * 128);
+                ++q_issued[qb];
+                for (int bx = 0; bx < C::NBOX; ++bx)
+                    ptx::tma_load_2d(sbase + C::OFF_Q + qb * C::Q_BYTES + bx * C::Q_BOX, &tm_q, bx * 64,
+                                     static_cast<int>(rb.q_row0), bar(C::B_QFULL + qb), pol_q);
+                for (int t = sg.t0; t < sg.t1; ++t, ++g) {
+                    const int st = g % C::STK;
+                    ok = wait_bar(bar(C::B_KEMPTY + st), ((g / C::STK) & 1) ^ 1, wmisc, p);
+                    if (!ok) break;
+                    ++k_issued[st];
+                    load_kv_tile<C>(p, &tm_k, sbase + C::OFF_K + st * C::KV_BYTES, bar(C::B_KFULL + st), rb, t, sg.n,
+                                    pol_kv);
+                }
+                ++seg_i;
+            }
+            for (int i = 0; i < C::STK; ++i) drain_bar(bar(C::B_KFULL + i), k_issued[i], p.timeout_cycles);
+            for (int i = 0; i < C::QBUF; ++i) drain_bar(bar(C::B_QFULL + i), q_issued[i], p.timeout_cycles);
+        }
+        // ------------------------------------------------------------ V producer
+        else if (warp == 1 && lane == 0) {
+            const uint64_t pol_kv = ptx::policy_evict_first();
+            SegWalker wk;
+            wk.init(p, misc->span, cta);
+            Seg sg;
+            uint32_t g = 0;
+            bool ok = true;
+            uint32_t v_issued[C::STV];
+            for (int i = 0; i < C::STV; ++i) v_issued[i] = 0;
+            while (ok && wk.next(p, sg)) {
+                if (sg.t1 <= sg.t0) continue;
+                const RB rb = rb_of(p, sg.w);
+                for (int t = sg.t0; t < sg.t1; ++t, ++g) {
+                    const int st = g % C::STV;
+                    ok = wait_bar(bar(C::B_VEMPTY + st), ((g / C::STV) & 1) ^ 1, wmisc, p);
+                    if (!ok) break;
+                    ++v_issued[st];
+                    load_kv_tile<C>(p, &tm_v, sbase + C::OFF_V + st * C::KV_BYTES, bar(C::B_VFULL + st), rb, t, sg.n,
+                                    pol_kv);
+                }
+            }
+            for (int i = 0; i < C::STV; ++i) drain_bar(bar(C::B_VFULL + i), v_issued[i], p.timeout_cycles);
+        }
+        // ------------------------------------------------------------ MMA issuer
+        else if (warp == 2 && lane == 0) {
+            SegWalker wk;
+            wk.init(p, misc->span, cta);
+            Seg sg;
+            int seg_i = 0;
+            uint32_t g = 0;
+            bool ok = true;
+            // S'(g) = K(g) Q^T: A = the K tile (M = keys, K-major), B = the 16-row Q tile (K-major)
+            auto issue_s = [&](uint32_t gg, uint32_t qbase, uint32_t kbase) {
+                const uint32_t d = tmem + C::TM_S + 16u * (gg & 1u);
+#pragma unroll
+                for (int kk = 0; kk < C::D / 16; ++kk) {
+                    const uint32_t off = (kk & 3) * 32;
+                    const uint64_t ad = ptx::umma_desc_sw128(kbase + (kk >> 2) * C::KV_BOX + off, 16, 1024);
+                    const uint64_t bd = ptx::umma_desc_sw128(qbase + (kk >> 2) * C::Q_BOX + off, 16, 1024);
+                    ptx::umma_bf16_ss(d, ad, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+                }
+                ptx::umma_commit(bar(C::B_SFULL + (gg & 1u)));
+            };
+            // O' (+)= V(gg)^T P'(gg): A = the V tile read MN-major (M = head dims), B = P'^T (K-major)
+            auto issue_pv = [&](uint32_t gg, bool first, int seg) -> bool {
+                const int st = gg % C::STV;
+                if (!wait_bar(bar(C::B_PFULL + (gg & 1u)), (gg >> 1) & 1u, wmisc, p)) return false;
+                if (!wait_bar(bar(C::B_VFULL + st), (gg / C::STV) & 1u, wmisc, p)) return false;
+                if (first && seg > 0 && !wait_bar(bar(C::B_OFREE), (seg - 1) & 1, wmisc, p)) return false;
+                ptx::tc_fence_after();
+                const uint32_t vbase = sbase + C::OFF_V + st * C::KV_BYTES;
+                const uint32_t pbase = sbase + C::OFF_P + (gg & 1u) * C::P_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                    const uint64_t ad = ptx::umma_desc_sw128(vbase + kk * 2048, C::KV_BOX, 1024);
+                    const uint64_t bd = ptx::umma_desc_sw128(pbase + (kk >> 2) * C::P_BOX + (kk & 3) * 32, 16, 1024);
+                    ptx::umma_bf16_ss(tmem + C::TM_O, ad, bd, C::IDESC_PV, (kk > 0 || !first) ? 1u : 0u);
+                }
+                ptx::umma_commit(bar(C::B_PVDONE + (gg & 1u)));
+                ptx::umma_commit(bar(C::B_VEMPTY + st));
+                return true;
+            };
+            bool have_prev = false, prev_first = false;
+            uint32_t prev_g = 0;
+            int prev_seg = 0;
+            while (ok && wk.next(p, sg)) {
+                if (sg.t1 <= sg.t0) continue;
+                // the previous segment's last PV' goes out before this segment's Q is awaited
+                if (have_prev) {
+                    ok = issue_pv(prev_g, prev_first, prev_seg);
+                    if (!ok) break;
+                    have_prev = false;
+                }
+                const int qb = seg_i % C::QBUF;
+                ok = wait_bar(bar(C::B_QFULL + qb), (seg_i / C::QBUF) & 1, wmisc, p);
+                if (!ok) break;
+                const uint32_t qbase = sbase + C::OFF_Q + qb * C::Q_BYTES;
+                for (int t = sg.t0; t < sg.t1 && ok; ++t, ++g) {
+                    const int stk = g % C::STK;
+                    ok = wait_bar(bar(C::B_KFULL + stk), (g / C::STK) & 1, wmisc, p);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    issue_s(g, qbase, sbase + C::OFF_K + stk * C::KV_BYTES);
+                    ptx::umma_commit(bar(C::B_KEMPTY + stk));
+                    if (t == sg.t1 - 1) ptx::umma_commit(bar(C::B_QEMPTY + qb));
+                    if (have_prev) {
+                        ok = issue_pv(prev_g, prev_first, prev_seg);
+                        if (!ok) break;
+                    }
+                    have_prev = true;
+                    prev_g = g;
+                    prev_first = (t == sg.t0);
+                    prev_seg = seg_i;
+                }
+                ++seg_i;
+            }
+            if (ok && have_prev) ok = issue_pv(prev_g, prev_first, prev_seg);
+            ptx::umma_commit(bar(C::B_FINAL));
+            drain_bar(bar(C::B_FINAL), 1, p.timeout_cycles);
+        }
+        // ------------------------------------------------------------ ticket taker
+        else if (warp == 3 && lane == 0) {
+            SegWalker wk;
+            wk.init(p, misc->span, cta);
+            Seg sg;
+            int j = 0;
+            const long long tot = misc->span.tot;
+            while (j < 2 && wk.next(p, sg)) {
+                if (sg.kind != 1) continue;
+                if (!wait_bar(bar(C::B_MJOB + j), 0, wmisc, p)) break;
+                const int c_first = cta_of(sg.pw, tot, NC);
+                const int c_last = cta_of(sg.pw + sg.ntiles - 1, tot, NC);
+                int ncontrib = 0;
+                for (int cc = c_first; cc <= c_last; ++cc) ncontrib += span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC);
+                __threadfence();
+                const int old = atomicAdd(p.counters + sg.w, 1);
+                misc->ticket[j] = (old == ncontrib - 1);
+                ptx::mbar_arrive(bar(C::B_MTICK + j));
+                ++j;
+            }
+        }
+    }
+    // ---------------------------------------------------------------- softmax warps
+    else {
+        const int quad = warp & 3;
+        const int kl = quad * 32 + lane;  // key of the tile = S' lane; head dim = O' lane
+        const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+        const int stid = threadIdx.x - 128;
+        uint32_t rph = 0, xph = 0;
+        auto xsync = [&]() -> bool {  // the four softmax warps, bounded
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(C::B_XSYNC));
+            const bool r = wait_bar(bar(C::B_XSYNC), xph & 1, wmisc, p);
+            ++xph;
+            ptx::tc_fence_after();
+            return __all_sync(0xffffffffu, r);
+        };
+        // reduce NR values per thread over all 128 keys of the softmax warps
+        auto cta_reduce = [&](const float (&x)[NR], float (&out)[NR], bool is_max) -> bool {
+            const float wv = is_max ? dec_warp_reduce<NR, true>(x, lane) : dec_warp_reduce<NR, false>(x, lane);
+            float(*red)[4] = misc->red[rph & 1];
+            if (dec_row_writer<NR>(lane)) red[dec_row_of<NR>(lane)][quad] = wv;
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(C::B_RED));
+            bool okr = wait_bar(bar(C::B_RED), rph & 1, wmisc, p);
+            ++rph;
+            okr = __all_sync(0xffffffffu, okr);
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const float4 w4 = *reinterpret_cast<const float4*>(&red[r][0]);
+                out[r] = is_max ? fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w)) : (w4.x + w4.y) + (w4.z + w4.w);
+            }
+            return okr;
+        };
+        SegWalker wk;
+        wk.init(p, misc->span, cta);
+        Seg sg;
+        uint32_t g = 0;
+        bool ok = true;
+        int njob = 0;
+        int seg_i = 0;
+        // P'^T address of this thread's key in a P' buffer: row r adds r*128 and
+        // swizzles the 16-byte chunk by r % 8
+        const int pkey_box = kl >> 6, pkey_chunk = (kl & 63) >> 3, pkey_in = (kl & 7) * 2;
+
+        while (ok && wk.next(p, sg)) {
+            if (sg.t1 <= sg.t0) continue;
+            const RB rb = rb_of(p, sg.w);
+            // visible keys of each packed row: key <= lim[r] (-1: row absent)
+            int lim[NR];
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                int l = -1;
+                if (r < rb.rows_valid) {
+                    const int i = r % p.Tq;
+                    l = p.causal ? (sg.n - p.Tq + i) : (sg.n - 1);
+                    if (l > sg.n - 1) l = sg.n - 1;
+                }
+                lim[r] = l;
+            }
+            float m_run[NR], l_t[NR];
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                m_run[r] = -INFINITY;
+                l_t[r] = 0.f;
+            }
+            for (int t = sg.t0; t < sg.t1; ++t, ++g) {
+                const bool first = (t == sg.t0);
+                ok = wait_bar(bar(C::B_SFULL + (g & 1u)), (g >> 1) & 1u, wmisc, p);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                float x[NR];
+                {
+                    uint32_t sr[NR];
+                    const uint32_t ts = tmem + lane_off + C::TM_S + 16u * (g & 1u);
+                    if constexpr (NR == 16) ptx::tmem_ld16(ts, sr);
+                    else ptx::tmem_ld8(ts, sr);
+                    ptx::tmem_wait_ld();
+                    const int key = t * C::BN + kl;
+                    // mask by selection (never by adding -inf: NaN + -inf stays NaN)
+#pragma unroll
+                    for (int r = 0; r < NR; ++r) x[r] = (key <= lim[r]) ? __uint_as_float(sr[r]) * p.scale_log2 : -INFINITY;
+                }
+                float mt[NR];
+                ok = cta_reduce(x, mt, true);
+                if (!ok) break;
+                // online softmax with a lazy rescale: the reference max moves only
+                // when a row's max grows by more than 2^8
+                bool grow = false;
+#pragma unroll
+                for (int r = 0; r < NR; ++r) grow |= mt[r] > m_run[r] + RESCALE_THRESHOLD;
+                if (grow) {
+                    float alpha[NR];
+#pragma unroll
+                    for (int r = 0; r < NR; ++r) {
+                        const float mn = fmaxf(m_run[r], mt[r]);
+                        alpha[r] = (m_run[r] == -INFINITY) ? 0.f : ptx::ex2(m_run[r] - mn);
+                        l_t[r] *= alpha[r];
+                        m_run[r] = mn;
+                    }
+                    if (!first) {
+                        // O' holds PV'(g-1) once it completes; scale column r by alpha[r]
+                        bool okw = wait_bar(bar(C::B_PVDONE + ((g - 1) & 1u)), ((g - 1) >> 1) & 1u, wmisc, p);
+                        okw = __all_sync(0xffffffffu, okw);
+                        if (!okw) { ok = false; break; }
+                        ptx::tc_fence_after();
+                        const uint32_t to = tmem + lane_off + C::TM_O;
+                        uint32_t o[NR];
+                        if constexpr (NR == 16) ptx::tmem_ld16(to, o);
+                        else ptx::tmem_ld8(to, o);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int r = 0; r < NR; ++r) o[r] = __float_as_uint(__uint_as_float(o[r]) * alpha[r]);
+                        if constexpr (NR == 16) ptx::tmem_st16(to, o);
+                        else ptx::tmem_st8(to, o);
+                        ptx::tmem_wait_st();
+                    }
+                }
+                // P' buffer g % 2 was last read by PV'(g-2)
+                if (g >= 2) {
+                    bool okw = wait_bar(bar(C::B_PVDONE + (g & 1u)), ((g - 2) >> 1) & 1u, wmisc, p);
+                    okw = __all_sync(0xffffffffu, okw);
+                    if (!okw) { ok = false; break; }
+                }
+                uint8_t* pb = smem + C::OFF_P + (g & 1u) * C::P_BYTES + pkey_box * C::P_BOX + pkey_in;
+#pragma unroll
+                for (int r = 0; r < NR; ++r) {
+                    const float mu = (m_run[r] == -INFINITY) ? 0.f : m_run[r];
+                    const float pr = ptx::ex2(x[r] - mu);
+                    l_t[r] += pr;
+                    *reinterpret_cast<__nv_bfloat16*>(pb + r * 128 + ((pkey_chunk ^ (r & 7)) << 4)) = __float2bfloat16_rn(pr);
+                }
+                // padded key rows of the V tile reach the MMA as zeros (0 * NaN = NaN)
+                if ((t + 1) * C::BN > sg.n) {
+                    const int st = g % C::STV;
+                    bool okv = wait_bar(bar(C::B_VFULL + st), (g / C::STV) & 1, wmisc, p);
+                    okv = __all_sync(0xffffffffu, okv);
+                    if (!okv) { ok = false; break; }
+                    if (t * C::BN + kl >= sg.n) {
+                        uint8_t* vt = smem + C::OFF_V + st * C::KV_BYTES + kl * 128;
+#pragma unroll
+                        for (int bx = 0; bx < C::NBOX; ++bx)
+#pragma unroll
+                            for (int c = 0; c < 8; ++c)
+                                *reinterpret_cast<uint4*>(vt + bx * C::KV_BOX + c * 16) = make_uint4(0, 0, 0, 0);
+                    }
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar(C::B_PFULL + (g & 1u)));
+            }
+            if (!ok) break;
+
+            // ------------------------------------------------ segment epilogue
+            {
+                bool okw = wait_bar(bar(C::B_PVDONE + ((g - 1) & 1u)), ((g - 1) >> 1) & 1u, wmisc, p);
+                okw = __all_sync(0xffffffffu, okw);
+                if (!okw) { ok = false; break; }
+                ptx::tc_fence_after();
+            }
+            float lsum[NR];
+            ok = cta_reduce(l_t, lsum, false);
+            if (!ok) break;
+            uint32_t o[NR];
+            {
+                const uint32_t to = tmem + lane_off + C::TM_O;
+                if constexpr (NR == 16) ptx::tmem_ld16(to, o);
+                else ptx::tmem_ld8(to, o);
+                ptx::tmem_wait_ld();
+            }
+            // O' is read: the next segment's first PV' may overwrite it
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(C::B_OFREE));
+            const bool direct = (sg.kind == 0);
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                if (r >= rb.rows_valid) break;
+                const long long fr = rb.q_row0 + r;  // flat row (b*Hq + h)*Tq + i
+                float w = 0.f, lse_v = -INFINITY;
+                if (direct) {
+                    const int h = rb.g * p.G + r / p.Tq;
+                    const float sk = (p.sink != nullptr) ? __ldg(p.sink + h) * LOG2E : -INFINITY;
+                    const float M = fmaxf(m_run[r], sk);
+                    if (M != -INFINITY) {
+                        const float a = (lsum[r] > 0.f) ? ptx::ex2(m_run[r] - M) : 0.f;
+                        const float lt = lsum[r] * a + ((sk != -INFINITY) ? ptx::ex2(sk - M) : 0.f);
+                        if (lt > 0.f) {
+                            w = a / lt;
+                            lse_v = (M + __log2f(lt)) * LN2;
+                        }
+                    }
+                    p.out[fr * C::D + kl] = __float2bfloat16_rn(w != 0.f ? __uint_as_float(o[r]) * w : 0.f);
+                    if (kl == 0 && p.lse != nullptr) p.lse[fr] = lse_v;
+                } else {
+                    if (lsum[r] > 0.f) {
+                        w = 1.f / lsum[r];
+                        lse_v = (m_run[r] + __log2f(lsum[r])) * LN2;
+                    }
+                    const long long prow = static_cast<long long>(sg.slot) * BM + r;
+                    __stcg(p.part_o + prow * C::D + kl, w != 0.f ? __uint_as_float(o[r]) * w : 0.f);
+                    if (kl == 0) __stcg(p.part_lse + prow, lse_v);
+                }
+            }
+            // a split segment's partial rows are written
+            if (!xsync()) { ok = false; break; }
+            if (sg.kind == 1 && njob < 2) {
+                if (stid == 0) {
+                    misc->jobs[njob] = sg;
+                    ptx::mbar_arrive(bar(C::B_MJOB + njob));
+                }
+                ++njob;
+            }
+            ++seg_i;
+        }
+        // merges of the row-blocks whose last piece this CTA wrote
+        for (int j = 0; ok && j < njob; ++j) {
+            ok = wait_bar(bar(C::B_MTICK + j), 0, wmisc, p);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            if (!misc->ticket[j]) continue;
+            __threadfence();
+            const Seg sgm = misc->jobs[j];
+            const RB rb = rb_of(p, sgm.w);
+            const long long tot = misc->span.tot;
+            const int c_first = cta_of(sgm.pw, tot, NC);
+            const int c_last = cta_of(sgm.pw + sgm.ntiles - 1, tot, NC);
+            const bool c0_first = span_begin(c_first, tot, NC) == sgm.pw;
+            const long long RW = BM;
+            if (warp == 4) {
+                int nm = 0;
+                for (int base = c_first; base <= c_last; base += 32) {
+                    const int cc = base + lane;
+                    const bool has = cc <= c_last && span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC);
+                    const unsigned m = __ballot_sync(0xffffffffu, has);
+                    const int k = nm + __popc(m & ((1u << lane) - 1u));
+                    if (has && k < kMaxMergeSlots) misc->mslot[k] = static_cast<int>(merge_slot(cc, c_first, c0_first));
+                    nm += __popc(m);
+                }
+                if (lane == 0) misc->nmerge = nm;
+            }
+            if (!xsync()) { ok = false; break; }
+            const int nm = misc->nmerge;
+            auto slot_of = [&](int k) -> long long {  // k-th contributing CTA's slot
+                if (nm <= kMaxMergeSlots) return misc->mslot[k];
+                int seen = 0;
+                for (int cc = c_first; cc <= c_last; ++cc) {
+                    if (!(span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC))) continue;
+                    if (seen++ == k) return merge_slot(cc, c_first, c0_first);
+                }
+                return 0;
+            };
+            // lse of each merged row (the sink enters here, once); eight pieces' loads at a time
+            for (int r = stid; r < rb.rows_valid; r += NSOFT_DEC) {
+                const int hr = rb.g * p.G + r / p.Tq;
+                const float sk = (p.sink != nullptr) ? __ldg(p.sink + hr) : -INFINITY;
+                float Lx = sk, z = 0.f;
+                for (int k0 = 0; k0 < nm; k0 += 8) {
+                    float lv[8];
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj)
+                        lv[jj] = (k0 + jj < nm) ? __ldcg(p.part_lse + slot_of(k0 + jj) * RW + r) : -INFINITY;
+                    float mx = Lx;
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) mx = fmaxf(mx, lv[jj]);
+                    if (mx != -INFINITY) {
+                        // running (max, sum) over the pieces seen so far
+                        z = (Lx != -INFINITY) ? z * __expf(Lx - mx) : 0.f;
+#pragma unroll
+                        for (int jj = 0; jj < 8; ++jj) z += __expf(lv[jj] - mx);
+                        Lx = mx;
+                    }
+                }
+                float ltr = -INFINITY;
+                if (Lx != -INFINITY) {
+                    if (sk != -INFINITY) z += __expf(sk - Lx);
+                    ltr = Lx + __logf(z);
+                }
+                misc->mlse[r] = ltr;
+                if (p.lse != nullptr) p.lse[rb.q_row0 + r] = ltr;
+            }
+            if (!xsync()) { ok = false; break; }
+            // O rows: weight exp(lse_k - lse) per piece; thread = head dim; every
+            // row's loads of two pieces in flight together
+            float lt[NR], acc[NR];
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                lt[r] = (r < rb.rows_valid) ? misc->mlse[r] : -INFINITY;
+                acc[r] = 0.f;
+            }
+            for (int k0 = 0; k0 < nm; k0 += 2) {
+                float lw[2][NR], xv[2][NR];
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    const bool has = k0 + jj < nm;
+                    const long long sl = has ? slot_of(k0 + jj) : 0;
+#pragma unroll
+                    for (int r = 0; r < NR; ++r) {
+                        const bool live = has && lt[r] != -INFINITY;
+                        lw[jj][r] = live ? __ldcg(p.part_lse + sl * RW + r) : -INFINITY;
+                        xv[jj][r] = live ? __ldcg(p.part_o + (sl * RW + r) * C::D + kl) : 0.f;
+                    }
+                }
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+                    for (int r = 0; r < NR; ++r)
+                        if (lw[jj][r] != -INFINITY) acc[r] += __expf(lw[jj][r] - lt[r]) * xv[jj][r];
+            }
+#pragma unroll
+            for (int r = 0; r < NR; ++r)
+                if (r < rb.rows_valid) p.out[(rb.q_row0 + r) * C::D + kl] = __float2bfloat16_rn(acc[r]);
+            if (stid == 0) p.counters[sgm.w] = 0;
+            if (!xsync()) { ok = false; break; }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, C::TM_COLS);
+    }
+}
+
+}  // namespace gqa
+static_assert(sizeof(gqa::DecMisc) <= gqa::DecCfg<8>::MISC_BYTES, "misc block");

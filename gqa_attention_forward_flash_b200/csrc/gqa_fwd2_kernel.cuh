@@ -38,9 +38,10 @@ constexpr int NUM_THREADS2 = 384;  // 12 warps = 3 warpgroups
 constexpr int NSOFT2 = 256;        // softmax threads (two warpgroups)
 constexpr int kMaxMergeSlots = 64; // pieces a row-block's merge lists in shared memory
 
-template <int D_, int STK_, int STV_, int RBQ_>
+template <int D_, int STK_, int STV_, int RBQ_, bool PAGED_ = false>
 struct Fwd2Cfg {
     static constexpr int D = D_, BN = 128, STK = STK_, STV = STV_, RBQ = RBQ_;
+    static constexpr bool PAGED = PAGED_;  // K/V from a paged cache (chosen at compile time)
     static_assert(D == 64 || D == 128, "head dim");
     static constexpr int NBOX = D / 64;
     static constexpr int Q_BOX = BM * 128;
@@ -110,7 +111,7 @@ constexpr int PAGE_BATCH = 4;  // page ids fetched per batch of independent load
 template <class C>
 __device__ __forceinline__ void load_kv_tile(const Params& p, const CUtensorMap* tm, uint32_t dst, uint32_t full_bar,
                                              const RB& rb, int t, int n, uint64_t policy) {
-    if (p.page_size == 0) {
+    if constexpr (!C::PAGED) {
         ptx::mbar_arrive_expect_tx(full_bar, C::NBOX * p.kv_box_rows * 128);
         const int y = static_cast<int>(rb.kv_row0 + static_cast<long long>(t) * C::BN);
         for (int bx = 0; bx < C::NBOX; ++bx) ptx::tma_load_2d(dst + bx * C::KV_BOX, tm, bx * 64, y, full_bar, policy);

@@ -326,6 +326,131 @@ def _single_lane(segs, stk, stv, rnd):
     _simulate(bars, roles, rnd)
 
 
+# --------------------------------------------------------------------------
+# swap-AB decode kernel (head dim 128, at most 16 packed rows): gqa_dec_kernel
+
+
+def _decode(segs, stk, stv, rnd):
+    bars = {}
+
+    def mk(name, count):
+        bars[name] = _Bar(count)
+
+    for i in range(2):
+        mk("QF%d" % i, 1)
+        mk("QE%d" % i, 1)
+        mk("SF%d" % i, 1)
+        mk("PF%d" % i, 4)
+        mk("PD%d" % i, 1)
+        mk("MJ%d" % i, 1)
+        mk("MT%d" % i, 1)
+    for i in range(stk):
+        mk("KF%d" % i, 1)
+        mk("KE%d" % i, 1)
+    for i in range(stv):
+        mk("VF%d" % i, 1)
+        mk("VE%d" % i, 1)
+    mk("OFREE", 4)
+    mk("RED", 4)
+    mk("X", 4)
+    # decisions every softmax warp takes alike (they follow the CTA-wide row maxima)
+    grow = [[rnd.random() < 0.3 for _ in range(n)] for n, _ in segs]
+    tail = [[rnd.random() < 0.3 for _ in range(n)] for n, _ in segs]
+    merges = [rnd.random() < 0.5 for _ in segs]
+    nsplit = min(2, sum(1 for _, k in segs if k == 1))
+
+    def kprod():
+        g = 0
+        for si, (n, _) in enumerate(segs):
+            yield ("wait", "QE%d" % (si % 2), si // 2 - 1)
+            yield ("tma", ["QF%d" % (si % 2)])
+            for _ in range(n):
+                yield ("wait", "KE%d" % (g % stk), g // stk - 1)
+                yield ("tma", ["KF%d" % (g % stk)])
+                g += 1
+
+    def vprod():
+        g = 0
+        for n, _ in segs:
+            for _ in range(n):
+                yield ("wait", "VE%d" % (g % stv), g // stv - 1)
+                yield ("tma", ["VF%d" % (g % stv)])
+                g += 1
+
+    def mma():
+        def pv(gg, first, seg):
+            yield ("wait", "PF%d" % (gg % 2), gg // 2)
+            yield ("wait", "VF%d" % (gg % stv), gg // stv)
+            if first and seg > 0:
+                yield ("wait", "OFREE", seg - 1)
+            yield ("mma", ["PD%d" % (gg % 2), "VE%d" % (gg % stv)])
+
+        g = 0
+        prev = None
+        for si, (n, _) in enumerate(segs):
+            if prev is not None:
+                yield from pv(*prev)
+                prev = None
+            yield ("wait", "QF%d" % (si % 2), si // 2)
+            for t in range(n):
+                yield ("wait", "KF%d" % (g % stk), g // stk)
+                yield ("mma", ["SF%d" % (g % 2), "KE%d" % (g % stk)] + (["QE%d" % (si % 2)] if t == n - 1 else []))
+                if prev is not None:
+                    yield from pv(*prev)
+                prev = (g, t == 0, si)
+                g += 1
+        if prev is not None:
+            yield from pv(*prev)
+
+    ph = {}
+
+    def softmax(w):
+        ph[w] = {"RED": 0, "X": 0}
+
+        def sync(name):
+            yield ("arrive", name)
+            yield ("wait", name, ph[w][name])
+            ph[w][name] += 1
+
+        g = 0
+        njob = 0
+        for si, (n, kind) in enumerate(segs):
+            for t in range(n):
+                yield ("wait", "SF%d" % (g % 2), g // 2)
+                yield from sync("RED")
+                if grow[si][t] and t > 0:
+                    yield ("wait", "PD%d" % ((g - 1) % 2), (g - 1) // 2)
+                if g >= 2:
+                    yield ("wait", "PD%d" % (g % 2), (g - 2) // 2)
+                if tail[si][t]:
+                    yield ("wait", "VF%d" % (g % stv), g // stv)
+                yield ("arrive", "PF%d" % (g % 2))
+                g += 1
+            yield ("wait", "PD%d" % ((g - 1) % 2), (g - 1) // 2)
+            yield from sync("RED")
+            yield ("arrive", "OFREE")
+            yield from sync("X")
+            if kind == 1 and njob < 2:
+                if w == 0:
+                    yield ("arrive", "MJ%d" % njob)
+                njob += 1
+        for j in range(njob):
+            yield ("wait", "MT%d" % j, 0)
+            if merges[j]:
+                for _ in range(3):
+                    yield from sync("X")
+
+    def tickets():
+        for j in range(nsplit):
+            yield ("wait", "MJ%d" % j, 0)
+            yield ("arrive", "MT%d" % j)
+
+    roles = {"kprod": kprod(), "vprod": vprod(), "mma": mma(), "tickets": tickets()}
+    for w in range(4):
+        roles["softmax%d" % w] = softmax(w)
+    _simulate(bars, roles, rnd)
+
+
 def _layouts(seed, count):
     rnd = random.Random(seed)
     for trial in range(count):
@@ -342,6 +467,11 @@ def test_two_lane_protocol_has_no_deadlock_or_aliasing(rbq):
 def test_single_lane_protocol_has_no_deadlock_or_aliasing():
     for trial, segs, stk, stv in _layouts(7, 400):
         _single_lane(segs, stk, stv, random.Random(trial))
+
+
+def test_decode_protocol_has_no_deadlock_or_aliasing():
+    for trial, segs, stk, stv in _layouts(5, 400):
+        _decode(segs, stk, stv, random.Random(trial))
 
 
 def test_model_catches_a_wrong_wait_index():
