@@ -23,13 +23,15 @@ STATUS = {
 MAX_SPLITS = 256
 
 # exported names and their C signatures (restype, argtypes)
-_P, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+_P, _I, _F, _L = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong
 SIGNATURES = {
     "gqa_attention_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "gqa_attention_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "gqa_attention_fwd_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "gqa_attention_fwd_partial": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P, _P]),
     "gqa_splitkv_combine": (_I, [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "gqa_shard_lengths": (_I, [_P, _I, _I, _I, _P, _P]),
+    "gqa_combine_shards": (_I, [_P, _L, _P, _L, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
     "gqa_get_device_error": (_I, [_P]),
     "gqa_profile_begin": (_I, []),
     "gqa_profile_take": (_I, [_P, _I, _P]),
@@ -184,6 +186,34 @@ def gqa_splitkv_combine(o_part, lse_part, sink=None, out=None, lse=None, stream=
     rc = load().gqa_splitkv_combine(_ptr(o_part), _ptr(lse_part), S, _ptr(sink), _ptr(out), _ptr(lse),
                                     B, Hq, Tq, d, _stream(stream))
     _check("gqa_splitkv_combine", rc)
+    return out, lse
+
+
+def gqa_shard_lengths(kv_lens, key_offset, shard_capacity, out=None, stream=None):
+    """clamp(kv_lens - key_offset, 0, shard_capacity): int32 [B] on the device."""
+    _need(kv_lens, torch.int32, "kv_lens", 1)
+    if out is None:
+        out = torch.empty_like(kv_lens)
+    rc = load().gqa_shard_lengths(_ptr(kv_lens), kv_lens.shape[0], int(key_offset), int(shard_capacity), _ptr(out),
+                                  _stream(stream))
+    _check("gqa_shard_lengths", rc)
+    return out
+
+
+def gqa_combine_shards(o_shards, lse_shards, sink=None, out=None, lse=None, stream=None):
+    """LSE merge of per-shard results: o_shards bf16 [S, B, Hq, Tq, d] (any shard
+    stride, rows contiguous), lse_shards fp32 [S, B, Hq, Tq].  Returns (out, lse)."""
+    S, B, Hq, Tq, d = o_shards.shape
+    assert o_shards.dtype == torch.bfloat16 and lse_shards.dtype == torch.float32
+    assert o_shards[0].is_contiguous() and lse_shards[0].is_contiguous()
+    assert tuple(lse_shards.shape) == (S, B, Hq, Tq)
+    if out is None:
+        out = torch.empty((B, Hq, Tq, d), dtype=torch.bfloat16, device=o_shards.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=o_shards.device)
+    rc = load().gqa_combine_shards(_ptr(o_shards), o_shards.stride(0), _ptr(lse_shards), lse_shards.stride(0), S,
+                                   _ptr(sink), _ptr(out), _ptr(lse), B, Hq, Tq, d, _stream(stream))
+    _check("gqa_combine_shards", rc)
     return out, lse
 
 

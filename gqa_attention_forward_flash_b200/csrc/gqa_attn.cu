@@ -475,6 +475,44 @@ extern "C" int gqa_splitkv_combine(const float* o_part, const float* lse_part, i
     return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
+extern "C" int gqa_shard_lengths(const int32_t* kv_lens, int B, int key_offset, int shard_capacity,
+                                 int32_t* shard_lens, gqa_stream_t stream) {
+    if (B < 0 || key_offset < 0 || shard_capacity < 0) return GQA_ERR_SHAPE;
+    if (B == 0) return GQA_OK;
+    if (!kv_lens || !shard_lens) return GQA_ERR_NULL;
+    const int blocks = (B + 255) / 256 < 1024 ? (B + 255) / 256 : 1024;
+    gqa_shard_lengths_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(kv_lens, B, key_offset,
+                                                                                      shard_capacity, shard_lens);
+    return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+extern "C" int gqa_combine_shards(const void* o_shards, long long o_shard_stride, const float* lse_shards,
+                                  long long lse_shard_stride, int num_shards, const float* sink, void* out, float* lse,
+                                  int B, int Hq, int Tq, int d, gqa_stream_t stream) {
+    if (B < 0 || Hq <= 0 || Tq < 0 || d <= 0 || d % 4 != 0) return GQA_ERR_SHAPE;
+    if (num_shards < 1 || num_shards > GQA_MAX_SPLITS) return GQA_ERR_SPLITS;
+    if (B == 0 || Tq == 0) return GQA_OK;
+    if (!o_shards || !lse_shards || !out) return GQA_ERR_NULL;
+    const long long rows = static_cast<long long>(B) * Hq * Tq;
+    if (num_shards > 1 && (o_shard_stride < rows * d || lse_shard_stride < rows)) return GQA_ERR_SHAPE;
+    // four bf16 (8 bytes) per load: the shards' starts stay 8-byte aligned
+    if (!aligned16(o_shards) || (o_shard_stride & 3) != 0 || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(lse_shards) & 3u))
+        return GQA_ERR_ALIGN;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState* s = nullptr;
+    int rc = get_state(&s);
+    if (rc) return rc;
+    long long blocks = (rows + 7) / 8;
+    const long long cap = static_cast<long long>(s->sm_count) * 16;
+    if (blocks > cap) blocks = cap;
+    const size_t smem = static_cast<size_t>(8) * num_shards * sizeof(float);
+    gqa_combine_shards_kernel<<<static_cast<int>(blocks), 256, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const __nv_bfloat16*>(o_shards), o_shard_stride, lse_shards, lse_shard_stride, num_shards, sink,
+        reinterpret_cast<__nv_bfloat16*>(out), lse, rows, Hq, Tq, d);
+    return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
 extern "C" int gqa_profile_begin(void) {
     std::lock_guard<std::mutex> lk(g_mu);
     int dev = 0;

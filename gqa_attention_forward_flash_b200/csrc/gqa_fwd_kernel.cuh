@@ -1166,6 +1166,68 @@ gqa_combine_uniform_kernel(const float* __restrict__ o_part, const float* __rest
     }
 }
 
+// ------------------------------------------------------------------ key shards
+// Sequence parallelism over a key-sharded K/V cache: the rank that holds keys
+// [key_offset, key_offset + capacity) of every sequence sees min(n, ...) of them.
+__global__ void gqa_shard_lengths_kernel(const int* __restrict__ kv_lens, int B, int key_offset, int capacity,
+                                         int* __restrict__ shard_lens) {
+    for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < B; b += gridDim.x * blockDim.x) {
+        const long long n = static_cast<long long>(kv_lens[b]) - key_offset;
+        shard_lens[b] = static_cast<int>(n < 0 ? 0 : (n > capacity ? capacity : n));
+    }
+}
+
+// LSE merge of per-shard results: shard s holds, for every row, its output over
+// the shard's keys (bf16, normalised) and that sum's lse (-inf: no visible key);
+// shard s of the outputs starts s * o_stride elements after the first, of the
+// lse s * l_stride elements after.  One warp per output row; the sink enters
+// once, here.
+__global__ void __launch_bounds__(256)
+gqa_combine_shards_kernel(const __nv_bfloat16* __restrict__ o_sh, long long o_stride, const float* __restrict__ l_sh,
+                          long long l_stride, int S, const float* __restrict__ sink, __nv_bfloat16* __restrict__ out,
+                          float* __restrict__ lse, long long rows, int Hq, int Tq, int d) {
+    extern __shared__ float wsh[];  // [8 warps][S]
+    const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float* wts = wsh + wib * S;
+    const long long nwarps = static_cast<long long>(gridDim.x) * 8;
+    for (long long row = static_cast<long long>(blockIdx.x) * 8 + wib; row < rows; row += nwarps) {
+        const int h = static_cast<int>((row / Tq) % Hq);
+        const float sk = (sink != nullptr) ? sink[h] : -INFINITY;
+        float L = sk;
+        for (int s = lane; s < S; s += 32) L = fmaxf(L, l_sh[s * l_stride + row]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L = fmaxf(L, __shfl_xor_sync(0xffffffffu, L, o));
+        float lt = -INFINITY;
+        if (L != -INFINITY) {
+            float z = 0.f;
+            for (int s = lane; s < S; s += 32) z += __expf(l_sh[s * l_stride + row] - L);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+            if (sink != nullptr) z += __expf(sk - L);
+            lt = L + __logf(z);
+        }
+        for (int s = lane; s < S; s += 32) wts[s] = (lt == -INFINITY) ? 0.f : __expf(l_sh[s * l_stride + row] - lt);
+        __syncwarp();
+        for (int c4 = lane; c4 < d / 4; c4 += 32) {
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            for (int s = 0; s < S; ++s) {
+                const float wgt = wts[s];
+                if (wgt == 0.f) continue;
+                const uint2 raw = *reinterpret_cast<const uint2*>(o_sh + s * o_stride + row * d + 4 * c4);
+                const __nv_bfloat162 x01 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+                const __nv_bfloat162 x23 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+                a0 += wgt * __low2float(x01);
+                a1 += wgt * __high2float(x01);
+                a2 += wgt * __low2float(x23);
+                a3 += wgt * __high2float(x23);
+            }
+            *reinterpret_cast<uint2*>(out + row * d + 4 * c4) = make_uint2(pack_bf16x2(a0, a1), pack_bf16x2(a2, a3));
+        }
+        if (lane == 0 && lse != nullptr) lse[row] = lt;
+        __syncwarp();
+    }
+}
+
 }  // namespace gqa
 
 static_assert(sizeof(gqa::Misc) <= 1664, "misc block");

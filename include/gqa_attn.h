@@ -119,6 +119,41 @@ int gqa_splitkv_combine(const float *o_part, const float *lse_part, int num_spli
                         gqa_stream_t stream);
 
 /*
+ * Sequence parallelism over a key-sharded K/V cache (kernbench2 benches commit
+ * log, long-context decode commit: each device holds a slice of every
+ * sequence's keys, computes the softmax state over its slice, and the states
+ * are merged).  A rank that holds keys [key_offset, key_offset + shard_capacity)
+ * of every sequence runs gqa_attention_fwd on its shard with the lengths below
+ * (no sink, causal = 0: with one query row per head, Tq = 1, causal and
+ * non-causal coincide), and gqa_combine_shards merges the ranks' results.
+ */
+
+/*
+ * shard_lens[b] = clamp(kv_lens[b] - key_offset, 0, shard_capacity): how many
+ * of sequence b's keys the shard holds.  kv_lens, shard_lens: int32 [B], device,
+ * caller-owned.  Errors: GQA_ERR_SHAPE (negative sizes), GQA_ERR_NULL.
+ */
+int gqa_shard_lengths(const int32_t *kv_lens, int B, int key_offset, int shard_capacity,
+                      int32_t *shard_lens, gqa_stream_t stream);
+
+/*
+ * LSE merge of per-shard results.  Shard s (0 <= s < num_shards) holds, for
+ * every row (b, h, i), its output over the shard's keys, normalised over them
+ * (bf16, o_shards + s * o_shard_stride elements, [B, Hq, Tq, d] contiguous) and
+ * that sum's log-sum-exp (fp32, lse_shards + s * lse_shard_stride elements,
+ * [B, Hq, Tq]; -inf, with output 0, where the shard holds no visible key):
+ *   lse = ln( sum_s exp(lse_s) + exp(sink[h]) ),   out = sum_s exp(lse_s - lse) * O_s
+ * (bf16, round to nearest).  The layout is what an all-gather of the ranks'
+ * (out, lse) buffers gives.  sink may be NULL; lse may be NULL.  Requires
+ * o_shards and out 16-byte aligned, o_shard_stride a multiple of 4 and, for
+ * num_shards > 1, strides that keep the shards from overlapping (else
+ * GQA_ERR_ALIGN / GQA_ERR_SHAPE); num_shards in [1, GQA_MAX_SPLITS].
+ */
+int gqa_combine_shards(const void *o_shards, long long o_shard_stride, const float *lse_shards,
+                       long long lse_shard_stride, int num_shards, const float *sink, void *out,
+                       float *lse, int B, int Hq, int Tq, int d, gqa_stream_t stream);
+
+/*
  * gqa_attention_fwd over a paged K/V cache (AstrAI commit log, attention
  * commits: a KV-source policy selecting contiguous or paged K/V, page-table and
  * cache-location indices stored as int32, the paged decode address path).  The
