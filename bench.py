@@ -301,13 +301,14 @@ def run_ours(args, w, ws, rank, local):
         kc, vc, table, lens = (t.to(dev) for t in paged_inputs(w, inp, args.page_size))
         del k, v
 
-    def step():
+    def step(st=None):
+        st = stream if st is None else st
         if args.page_size:
             binding.gqa_attention_fwd_paged(q, kc, vc, table, lens, sink, out, lse, scale=inp.scale,
-                                            causal=inp.causal, stream=stream)
+                                            causal=inp.causal, stream=st)
         else:
             binding.gqa_attention_fwd(q, k, v, kv, sink, out, lse, scale=inp.scale, causal=inp.causal,
-                                      stream=stream)
+                                      stream=st)
 
     for _ in range(args.warmup):
         step()
@@ -362,6 +363,9 @@ def run_ours(args, w, ws, rank, local):
                 "kernel": main_kernel_name(w), "kernel_ms": main_avg, "launches_per_step": launches_per_call(w),
                 "algorithmic_bytes": nbytes, "algorithmic_flops": nflops}
 
+    # back-to-back calls replayed from one CUDA graph (reported beside the timed steps)
+    graph = graph_timing(args, w, step, dev, nbytes, nflops) if args.graph > 0 else None
+
     # end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -380,7 +384,38 @@ def run_ours(args, w, ws, rank, local):
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": len(main_ms) * launches_per_call(w),
             "clocks": clocks,
         }
+        if graph is not None:
+            line["graph"] = graph
         print(json.dumps(line), flush=True)
+
+
+def graph_timing(args, w, step, dev, nbytes, nflops):
+    """args.graph calls captured back to back in one CUDA graph and replayed: the
+    time per call without host launch overhead, the way a layer loop replays a
+    captured decode step.  No L2 flush between the calls (a small workload's
+    inputs stay in L2), so this is a latency figure beside the timed steps, not
+    the headline value."""
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(args.graph):
+                step(s)
+    torch.cuda.synchronize(dev)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize(dev)
+    reps = 20
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) * 1e3 / (reps * args.graph)
+    return {"calls_per_graph": args.graph, "replays": reps, "us_per_call": us,
+            "value": throughput(w, nbytes, nflops, us / 1e6), "l2": "not flushed between calls"}
 
 
 def run_e2e(args, w, inp, dev, stream, nbytes, nflops, ws):
@@ -499,6 +534,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-step-seconds", type=float, default=3.0)
     ap.add_argument("--burn-seconds", type=float, default=1.5)
+    ap.add_argument("--graph", type=int, default=0,
+                    help="also time this many back-to-back calls captured in one CUDA graph")
     ap.add_argument("--page-size", type=int, default=0,
                     help="read K/V through gqa_attention_fwd_paged from a cache of pages of this many tokens "
                          "(0: contiguous K/V through gqa_attention_fwd)")

@@ -344,6 +344,14 @@ int run_streamk(Params& p, const void* q, const void* k, const void* v, DeviceSt
     const size_t slot_o = slot_rows * (d / ds) * sizeof(float);
     const size_t slot_l = (slot_rows * sizeof(float) + 255) & ~static_cast<size_t>(255);
     const size_t jobs = static_cast<size_t>(p.W) * ds * sizeof(CJob);
+    cudaStream_t st0 = reinterpret_cast<cudaStream_t>(stream);
+    if (s->scratch_bytes < slot_o + slot_l + jobs || s->counters_len < p.W * ds + 2) {
+        // growing the scratch allocates (and synchronises): not while the stream is
+        // being captured into a CUDA graph
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(st0, &cs) != cudaSuccess) return GQA_ERR_CUDA;
+        if (cs != cudaStreamCaptureStatusNone) return GQA_ERR_SCRATCH;
+    }
     rc = ensure_scratch(*s, slot_o + slot_l + jobs);
     if (rc) return rc;
     rc = ensure_counters(*s, p.W * ds + 2);
@@ -579,7 +587,9 @@ extern "C" const char* gqa_status_string(int status) {
         case GQA_ERR_UNSUPPORTED: return "unsupported head dim or GPU";
         case GQA_ERR_KVLEN: return "a kv_lens value was outside [0, Tkv] and was clamped";
         case GQA_ERR_PAGE: return "a page id was outside [0, num_pages); page 0 was read instead";
-        case GQA_ERR_SCRATCH: return "the problem needs more scratch than the fixed allocation-free array holds";
+        case GQA_ERR_SCRATCH:
+            return "the problem needs more scratch than is in place (the allocation-free array, or a call being "
+                   "captured into a CUDA graph before an uncaptured call of that size)";
         default: return "unknown status";
     }
 }

@@ -75,7 +75,7 @@ typedef enum {
     GQA_ERR_TIMEOUT = -6,     /* a bounded wait inside a kernel ran out (device-reported) */
     GQA_ERR_UNSUPPORTED = -7, /* head dim not in {64,128,256,512}, or the GPU is not sm_100 */
     GQA_ERR_KVLEN = -8,       /* a kv_lens value was outside [0, Tkv] (device-reported, clamped) */
-    GQA_ERR_SCRATCH = -9,     /* gqa_attention_fwd_noalloc: the problem exceeds its fixed scratch */
+    GQA_ERR_SCRATCH = -9,     /* the problem exceeds the scratch in place (noalloc's fixed array; graph capture) */
     GQA_ERR_PAGE = -10        /* gqa_attention_fwd_paged: a page id outside [0, num_pages) (device-reported) */
 } gqa_status;
 
@@ -85,6 +85,12 @@ typedef enum {
  * The forward.  out and lse receive the attention defined above.  scale is the
  * logit multiplier (1/sqrt(d) in the usual case); causal != 0 enables the
  * bottom-right causal mask.
+ *
+ * CUDA graphs: once an uncaptured call of the same or larger sizes has run on
+ * the device (the library's scratch is then in place), calls may be captured
+ * into a graph and replayed; a captured call that would need more scratch
+ * returns GQA_ERR_SCRATCH instead of allocating.  The same holds for
+ * gqa_attention_fwd_paged; gqa_attention_fwd_noalloc never allocates.
  */
 int gqa_attention_fwd(const void *q, const void *k, const void *v, const int32_t *kv_lens,
                       const float *sink, void *out, float *lse, int B, int Hq, int Hkv, int Tq,
