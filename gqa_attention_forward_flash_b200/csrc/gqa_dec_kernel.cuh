@@ -129,6 +129,32 @@ __device__ __forceinline__ bool dec_row_writer(int lane) {
     return (NR == 8) ? (lane & 3) == 0 : (lane & 1) == 0;
 }
 
+// O' (+)= V(gg)^T P'(gg): A = the V tile read MN-major (M = head dims), B = P'^T
+// (K-major).  Not inlined: the MMA thread reaches it from three places, and one
+// shared copy is in the instruction cache after the first tile (a copy that first
+// runs at a segment switch would be fetched while every SM streams K/V).
+template <class C>
+__device__ __noinline__ bool dec_issue_pv(const Params& p, Misc* wmisc, uint32_t bar0, uint32_t sbase, uint32_t tmem,
+                                          uint32_t gg, bool first, int seg) {
+    auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
+    const int st = gg % C::STV;
+    if (!wait_bar(bar(C::B_PFULL + (gg & 1u)), (gg >> 1) & 1u, wmisc, p)) return false;
+    if (!wait_bar(bar(C::B_VFULL + st), (gg / C::STV) & 1u, wmisc, p)) return false;
+    if (first && seg > 0 && !wait_bar(bar(C::B_OFREE), (seg - 1) & 1, wmisc, p)) return false;
+    ptx::tc_fence_after();
+    const uint32_t vbase = sbase + C::OFF_V + st * C::KV_BYTES;
+    const uint32_t pbase = sbase + C::OFF_P + (gg & 1u) * C::P_BYTES;
+#pragma unroll
+    for (int kk = 0; kk < C::BN / 16; ++kk) {
+        const uint64_t ad = ptx::umma_desc_sw128(vbase + kk * 2048, C::KV_BOX, 1024);
+        const uint64_t bd = ptx::umma_desc_sw128(pbase + (kk >> 2) * C::P_BOX + (kk & 3) * 32, 16, 1024);
+        ptx::umma_bf16_ss(tmem + C::TM_O, ad, bd, C::IDESC_PV, (kk > 0 || !first) ? 1u : 0u);
+    }
+    ptx::umma_commit(bar(C::B_PVDONE + (gg & 1u)));
+    ptx::umma_commit(bar(C::B_VEMPTY + st));
+    return true;
+}
+
 template <class C>
 __global__ void __launch_bounds__(NUM_THREADS_DEC, 1)
 gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -283,22 +309,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             };
             // O' (+)= V(gg)^T P'(gg): A = the V tile read MN-major (M = head dims), B = P'^T (K-major)
             auto issue_pv = [&](uint32_t gg, bool first, int seg) -> bool {
-                const int st = gg % C::STV;
-                if (!wait_bar(bar(C::B_PFULL + (gg & 1u)), (gg >> 1) & 1u, wmisc, p)) return false;
-                if (!wait_bar(bar(C::B_VFULL + st), (gg / C::STV) & 1u, wmisc, p)) return false;
-                if (first && seg > 0 && !wait_bar(bar(C::B_OFREE), (seg - 1) & 1, wmisc, p)) return false;
-                ptx::tc_fence_after();
-                const uint32_t vbase = sbase + C::OFF_V + st * C::KV_BYTES;
-                const uint32_t pbase = sbase + C::OFF_P + (gg & 1u) * C::P_BYTES;
-#pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk) {
-                    const uint64_t ad = ptx::umma_desc_sw128(vbase + kk * 2048, C::KV_BOX, 1024);
-                    const uint64_t bd = ptx::umma_desc_sw128(pbase + (kk >> 2) * C::P_BOX + (kk & 3) * 32, 16, 1024);
-                    ptx::umma_bf16_ss(tmem + C::TM_O, ad, bd, C::IDESC_PV, (kk > 0 || !first) ? 1u : 0u);
-                }
-                ptx::umma_commit(bar(C::B_PVDONE + (gg & 1u)));
-                ptx::umma_commit(bar(C::B_VEMPTY + st));
-                return true;
+                return dec_issue_pv<C>(p, wmisc, bar0, sbase, tmem, gg, first, seg);
             };
             bool have_prev = false, prev_first = false;
             uint32_t prev_g = 0;
@@ -536,7 +547,18 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(bar(C::B_OFREE));
             const bool direct = (sg.kind == 0);
+            // The row loop is rolled: this code first runs while every SM streams K/V,
+            // and each of its instruction-cache lines is fetched then (fewer lines,
+            // shorter stall).  It reads copies of the row state, so the arrays the tile
+            // loop uses stay in registers.
+            float em[NR], el[NR], eo[NR];
 #pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                em[r] = m_run[r];
+                el[r] = lsum[r];
+                eo[r] = __uint_as_float(o[r]);
+            }
+#pragma unroll 1
             for (int r = 0; r < NR; ++r) {
                 if (r >= rb.rows_valid) break;
                 const long long fr = rb.q_row0 + r;  // flat row (b*Hq + h)*Tq + i
@@ -544,24 +566,24 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (direct) {
                     const int h = rb.g * p.G + r / p.Tq;
                     const float sk = (p.sink != nullptr) ? __ldg(p.sink + h) * LOG2E : -INFINITY;
-                    const float M = fmaxf(m_run[r], sk);
+                    const float M = fmaxf(em[r], sk);
                     if (M != -INFINITY) {
-                        const float a = (lsum[r] > 0.f) ? ptx::ex2(m_run[r] - M) : 0.f;
-                        const float lt = lsum[r] * a + ((sk != -INFINITY) ? ptx::ex2(sk - M) : 0.f);
+                        const float a = (el[r] > 0.f) ? ptx::ex2(em[r] - M) : 0.f;
+                        const float lt = el[r] * a + ((sk != -INFINITY) ? ptx::ex2(sk - M) : 0.f);
                         if (lt > 0.f) {
                             w = a / lt;
                             lse_v = (M + __log2f(lt)) * LN2;
                         }
                     }
-                    p.out[fr * C::D + kl] = __float2bfloat16_rn(w != 0.f ? __uint_as_float(o[r]) * w : 0.f);
+                    p.out[fr * C::D + kl] = __float2bfloat16_rn(w != 0.f ? eo[r] * w : 0.f);
                     if (kl == 0 && p.lse != nullptr) p.lse[fr] = lse_v;
                 } else {
-                    if (lsum[r] > 0.f) {
-                        w = 1.f / lsum[r];
-                        lse_v = (m_run[r] + __log2f(lsum[r])) * LN2;
+                    if (el[r] > 0.f) {
+                        w = 1.f / el[r];
+                        lse_v = (em[r] + __log2f(el[r])) * LN2;
                     }
                     const long long prow = static_cast<long long>(sg.slot) * BM + r;
-                    __stcg(p.part_o + prow * C::D + kl, w != 0.f ? __uint_as_float(o[r]) * w : 0.f);
+                    __stcg(p.part_o + prow * C::D + kl, w != 0.f ? eo[r] * w : 0.f);
                     if (kl == 0) __stcg(p.part_lse + prow, lse_v);
                 }
             }
