@@ -115,3 +115,22 @@ def test_paged_entry_rejects_bad_arguments_on_the_host(lib):
     assert paged(lib, d=256) == -7             # only head dims 64 and 128
     assert paged(lib, table=None) == -1        # page table required
     assert paged(lib, lens=None) == -1         # kv_lens required
+
+
+def test_shard_entry_points_reject_bad_arguments_on_the_host(lib):
+    s = lib.gqa_shard_lengths
+    assert s(P(16), -1, 0, 8, P(16), None) == -2          # negative batch
+    assert s(P(16), 2, -3, 8, P(16), None) == -2          # negative offset
+    assert s(P(16), 2, 0, -1, P(16), None) == -2          # negative capacity
+    assert s(None, 2, 0, 8, P(16), None) == -1
+    assert s(P(16), 0, 0, 8, None, None) == 0             # nothing to do
+    c = lib.gqa_combine_shards
+    rows_d = 1 * 4 * 2 * 64
+    assert c(P(16), rows_d, P(16), 8, 0, None, P(16), P(16), 1, 4, 2, 64, None) == -4      # no shard
+    assert c(P(16), rows_d, P(16), 8, 257, None, P(16), P(16), 1, 4, 2, 64, None) == -4    # too many
+    assert c(P(16), rows_d, P(16), 8, 2, None, P(16), P(16), 1, 4, 2, 66, None) == -2      # d % 4
+    assert c(P(16), rows_d - 4, P(16), 8, 2, None, P(16), P(16), 1, 4, 2, 64, None) == -2  # shards overlap
+    assert c(P(16), rows_d, P(16), 7, 2, None, P(16), P(16), 1, 4, 2, 64, None) == -2      # lse shards overlap
+    assert c(P(16), rows_d + 2, P(16), 8, 2, None, P(16), P(16), 1, 4, 2, 64, None) == -3  # stride not 8-byte
+    assert c(P(24), rows_d, P(16), 8, 2, None, P(16), P(16), 1, 4, 2, 64, None) == -3      # base misaligned
+    assert c(None, rows_d, P(16), 8, 2, None, P(16), P(16), 1, 4, 2, 64, None) == -1
