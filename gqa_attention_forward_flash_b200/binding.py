@@ -194,6 +194,7 @@ def gqa_shard_lengths(kv_lens, key_offset, shard_capacity, out=None, stream=None
     _need(kv_lens, torch.int32, "kv_lens", 1)
     if out is None:
         out = torch.empty_like(kv_lens)
+    _need(out, torch.int32, "out", 1)
     rc = load().gqa_shard_lengths(_ptr(kv_lens), kv_lens.shape[0], int(key_offset), int(shard_capacity), _ptr(out),
                                   _stream(stream))
     _check("gqa_shard_lengths", rc)
@@ -203,14 +204,20 @@ def gqa_shard_lengths(kv_lens, key_offset, shard_capacity, out=None, stream=None
 def gqa_combine_shards(o_shards, lse_shards, sink=None, out=None, lse=None, stream=None):
     """LSE merge of per-shard results: o_shards bf16 [S, B, Hq, Tq, d] (any shard
     stride, rows contiguous), lse_shards fp32 [S, B, Hq, Tq].  Returns (out, lse)."""
+    if o_shards.dim() != 5 or o_shards.dtype != torch.bfloat16 or not o_shards.is_cuda or not o_shards[0].is_contiguous():
+        raise ValueError("o_shards must be a CUDA bf16 [S, B, Hq, Tq, d] tensor with contiguous shards")
     S, B, Hq, Tq, d = o_shards.shape
-    assert o_shards.dtype == torch.bfloat16 and lse_shards.dtype == torch.float32
-    assert o_shards[0].is_contiguous() and lse_shards[0].is_contiguous()
-    assert tuple(lse_shards.shape) == (S, B, Hq, Tq)
+    if (lse_shards.dtype != torch.float32 or not lse_shards.is_cuda or tuple(lse_shards.shape) != (S, B, Hq, Tq)
+            or not lse_shards[0].is_contiguous()):
+        raise ValueError("lse_shards must be a CUDA fp32 [S, B, Hq, Tq] tensor with contiguous shards")
+    if sink is not None:
+        _need(sink, torch.float32, "sink", 1)
     if out is None:
         out = torch.empty((B, Hq, Tq, d), dtype=torch.bfloat16, device=o_shards.device)
     if lse is None:
         lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=o_shards.device)
+    _need(out, torch.bfloat16, "out", 4)
+    _need(lse, torch.float32, "lse", 3)
     rc = load().gqa_combine_shards(_ptr(o_shards), o_shards.stride(0), _ptr(lse_shards), lse_shards.stride(0), S,
                                    _ptr(sink), _ptr(out), _ptr(lse), B, Hq, Tq, d, _stream(stream))
     _check("gqa_combine_shards", rc)
