@@ -11,6 +11,13 @@ ragged kv_len ~ U[1, 16384], NaN padding), measured in GB/s of algorithmic
 bytes (K/V rows visible to some query row, plus Q, O and lse); prefill
 workloads are measured in TFLOP/s (4*d flops per visible query/key pair).
 
+By default the same run then times every other workload of the metric (tiny
+prefill, short-q/long-kv prefill, full causal prefill, wide-head sink decode)
+the same way, with fewer steps and a shorter oracle sample, and reports each in
+a "workloads" block of the one JSON line (value, roofline, cpu_baseline, e2e,
+clocks); --only keeps to --workload.  Step times are reported as mean (the
+value) and median.
+
 Multi-GPU: the path needs no exchange, so N GPUs run N independent replicas
 (weak scaling); `value` sums the work of all ranks over the slowest rank's time.
 
@@ -40,6 +47,8 @@ from gqa_attention_forward_flash_b200.synth import WORKLOADS, Workload, make_inp
 
 METRIC = "GQA fwd TFLOP/s (prefill) & KV HBM GB/s (decode), 1 B200, % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# nominal B200 figures (HGX HBM3e bandwidth, dense bf16 tensor rate), for context beside the measured peaks
+SPEC_PEAKS = {"hbm_gbs": 7700.0, "bf16_tflops": 2250.0}
 L2_FLUSH_BYTES = 256 << 20
 PREFILL = {"full_causal_prefill"}
 
@@ -283,7 +292,9 @@ def paged_inputs(w: Workload, inp, page_size: int):
     return kc, vc, table, lens
 
 
-def run_ours(args, w, ws, rank, local):
+def measure(args, w, ws, rank, local, steps, cpu_seconds, with_e2e=True):
+    """Time `steps` calls of the forward on workload w (inputs resident in HBM,
+    L2 flushed before each call); returns the numbers of one JSON line."""
     from gqa_attention_forward_flash_b200 import binding
     binding.load()
     dev = torch.device("cuda", local if ws > 1 else 0)
@@ -328,11 +339,11 @@ def run_ours(args, w, ws, rank, local):
             step()
         torch.cuda.synchronize(dev)
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     binding.gqa_profile_begin()
     barrier(ws)
     torch.cuda.synchronize(dev)
-    for i in range(args.steps):
+    for i in range(steps):
         flush.zero_()
         ev[i][0].record(stream)
         step()
@@ -346,46 +357,81 @@ def run_ours(args, w, ws, rank, local):
         raise RuntimeError("device error %d in the timed steps" % err)
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = all_max(ws, sum(step_ms))
-    ms_per_step = total_ms / args.steps
+    ms_per_step = total_ms / steps
     value = throughput(w, nbytes * ws, nflops * ws, ms_per_step / 1e3)
+    median_ms = all_max(ws, statistics.median(step_ms))
 
     peaks, peak_src = load_peaks()
     main_avg = all_max(ws, statistics.mean(main_ms)) if main_ms else float("nan")
+    main_med = all_max(ws, statistics.median(main_ms)) if main_ms else float("nan")
     if bound == "hbm":
         achieved = nbytes / (main_avg / 1e3) / 1e9
         peak = float(peaks["hbm_gbs"])
     else:
         achieved = nflops / (main_avg / 1e3) / 1e12
         peak = float(peaks["bf16_tflops"])
+    spec_peak = SPEC_PEAKS["hbm_gbs"] if bound == "hbm" else SPEC_PEAKS["bf16_tflops"]
     traffic = None if args.page_size else traffic_for(w)
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": traffic, "peak_source": peak_src + (" (burst)" if bound == "tensor" else ""),
-                "kernel": main_kernel_name(w), "kernel_ms": main_avg, "launches_per_step": launches_per_call(w),
+                "frac_of_spec": achieved / spec_peak, "spec_peak": spec_peak,
+                "kernel": main_kernel_name(w), "kernel_ms": main_avg, "kernel_ms_median": main_med,
+                "launches_per_step": launches_per_call(w),
                 "algorithmic_bytes": nbytes, "algorithmic_flops": nflops}
+    if w.name == "short_q_long_kv":
+        # bandwidth-bound by its intensity (128 flop/B, below the ridge), but the
+        # workload is a prefill: its tensor-core fraction too
+        tf = nflops / (main_avg / 1e3) / 1e12
+        roofline["tensor"] = {"achieved": tf, "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
+                              "frac": tf / float(peaks["bf16_tflops"])}
 
     # back-to-back calls replayed from one CUDA graph (reported beside the timed steps)
     graph = graph_timing(args, w, step, dev, nbytes, nflops) if args.graph > 0 else None
 
     # end to end through the public API with host buffers
     e2e = None
-    if not args.no_e2e:
+    if with_e2e and not args.no_e2e:
         e2e = run_e2e(args, w, inp, dev, stream, nbytes, nflops, ws)
 
     cpu = None
-    if ws == 1 and rank == 0 and not args.no_cpu_baseline:
-        val, desc, cores, _ = oracle_sample(w, inp, args.cpu_seconds)
+    if ws == 1 and rank == 0 and not args.no_cpu_baseline and cpu_seconds > 0:
+        val, desc, cores, _ = oracle_sample(w, inp, cpu_seconds)
         cpu = {"value": val, "unit": unit, "cores": cores, "kind": "oracle", "sample": desc}
+    del q, out, flush
+    res = {"value": value, "unit": unit, "ms_per_step": ms_per_step, "ms_per_step_mean": ms_per_step,
+           "ms_per_step_median": median_ms, "steps": steps, "roofline": roofline, "cpu_baseline": cpu,
+           "e2e": e2e, "gpu_launches": len(main_ms) * launches_per_call(w), "clocks": clocks,
+           "config": config_of(w, args.page_size)}
+    if graph is not None:
+        res["graph"] = graph
+    return res
 
+
+def run_ours(args, w, ws, rank, local):
+    head = measure(args, w, ws, rank, local, args.steps, args.cpu_seconds)
+    extra = {}
+    if args.all_workloads:
+        # the metric's other configurations, each timed the same way in this run
+        # (fewer steps and a shorter CPU sample, so that the whole run stays short)
+        for name in sorted(WORKLOADS):
+            if name == w.name:
+                continue
+            r = measure(args, WORKLOADS[name], ws, rank, local, args.workload_steps, args.workload_cpu_seconds)
+            torch.cuda.empty_cache()
+            extra[name] = r
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(w, args.page_size),
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": len(main_ms) * launches_per_call(w),
-            "clocks": clocks,
+            "metric": METRIC, "value": head["value"], "unit": head["unit"], "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "ms_per_step_median": head["ms_per_step_median"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": head["config"],
+            "roofline": head["roofline"], "cpu_baseline": head["cpu_baseline"], "e2e": head["e2e"],
+            "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
         }
-        if graph is not None:
-            line["graph"] = graph
+        if "graph" in head:
+            line["graph"] = head["graph"]
+        if extra:
+            line["workloads"] = extra
         print(json.dumps(line), flush=True)
 
 
@@ -525,7 +571,7 @@ def traffic_for(w: Workload):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="batched_decode", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -534,6 +580,12 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-step-seconds", type=float, default=3.0)
     ap.add_argument("--burn-seconds", type=float, default=1.5)
+    ap.add_argument("--only", dest="all_workloads", action="store_false",
+                    help="time only --workload (by default the other workloads follow in a 'workloads' block)")
+    ap.add_argument("--workload-steps", type=int, default=40,
+                    help="timed steps of each workload in the 'workloads' block")
+    ap.add_argument("--workload-cpu-seconds", type=float, default=3.0,
+                    help="oracle seconds of each workload in the 'workloads' block")
     ap.add_argument("--graph", type=int, default=0,
                     help="also time this many back-to-back calls captured in one CUDA graph")
     ap.add_argument("--page-size", type=int, default=0,

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libgqa_attn.so")
 STATUS = {
     0: "GQA_OK", -1: "GQA_ERR_NULL", -2: "GQA_ERR_SHAPE", -3: "GQA_ERR_ALIGN", -4: "GQA_ERR_SPLITS",
     -5: "GQA_ERR_CUDA", -6: "GQA_ERR_TIMEOUT", -7: "GQA_ERR_UNSUPPORTED", -8: "GQA_ERR_KVLEN",
-    -9: "GQA_ERR_SCRATCH", -10: "GQA_ERR_PAGE",
+    -9: "GQA_ERR_SCRATCH", -10: "GQA_ERR_PAGE", -11: "GQA_ERR_SMEM_ALIGN",
 }
 MAX_SPLITS = 256
 
@@ -149,6 +149,10 @@ def gqa_attention_fwd_noalloc(q, k, v, kv_lens=None, sink=None, out=None, lse=No
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=q.device)
+    if kv_lens is not None:
+        _need(kv_lens, torch.int32, "kv_lens", 1)
+    if sink is not None:
+        _need(sink, torch.float32, "sink", 1)
     if scale is None:
         scale = d ** -0.5
     rc = load().gqa_attention_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_lens), _ptr(sink), _ptr(out),
@@ -161,12 +165,21 @@ def gqa_attention_fwd_noalloc(q, k, v, kv_lens=None, sink=None, out=None, lse=No
 def gqa_attention_fwd_partial(q, k, v, kv_lens=None, scale=None, causal=False, num_splits=2, o_part=None,
                               lse_part=None, stream=None):
     """Split partials (no combine, no sink): o_part fp32 [B,Hq,Tq,S,d], lse_part fp32 [B,Hq,Tq,S]."""
+    _need(q, torch.bfloat16, "q", 4)
+    _need(k, torch.bfloat16, "k", 4)
+    _need(v, torch.bfloat16, "v", 4)
+    if kv_lens is not None:
+        _need(kv_lens, torch.int32, "kv_lens", 1)
     B, Hq, Tq, d = q.shape
     _, Hkv, Tkv, _ = k.shape
     if o_part is None:
         o_part = torch.empty((B, Hq, Tq, num_splits, d), dtype=torch.float32, device=q.device)
     if lse_part is None:
         lse_part = torch.empty((B, Hq, Tq, num_splits), dtype=torch.float32, device=q.device)
+    _need(o_part, torch.float32, "o_part", 5)
+    _need(lse_part, torch.float32, "lse_part", 4)
+    if tuple(o_part.shape) != (B, Hq, Tq, num_splits, d) or tuple(lse_part.shape) != (B, Hq, Tq, num_splits):
+        raise ValueError("o_part must be [B, Hq, Tq, num_splits, d] and lse_part [B, Hq, Tq, num_splits]")
     if scale is None:
         scale = d ** -0.5
     rc = load().gqa_attention_fwd_partial(_ptr(q), _ptr(k), _ptr(v), _ptr(kv_lens), B, Hq, Hkv, Tq, Tkv, d,
@@ -178,11 +191,19 @@ def gqa_attention_fwd_partial(q, k, v, kv_lens=None, scale=None, causal=False, n
 
 def gqa_splitkv_combine(o_part, lse_part, sink=None, out=None, lse=None, stream=None):
     """LSE combine of [B,Hq,Tq,S,d] partials into bf16 out [B,Hq,Tq,d] and lse."""
+    _need(o_part, torch.float32, "o_part", 5)
+    _need(lse_part, torch.float32, "lse_part", 4)
     B, Hq, Tq, S, d = o_part.shape
+    if tuple(lse_part.shape) != (B, Hq, Tq, S):
+        raise ValueError("lse_part must be [B, Hq, Tq, S] for o_part [B, Hq, Tq, S, d]")
+    if sink is not None:
+        _need(sink, torch.float32, "sink", 1)
     if out is None:
         out = torch.empty((B, Hq, Tq, d), dtype=torch.bfloat16, device=o_part.device)
     if lse is None:
         lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=o_part.device)
+    _need(out, torch.bfloat16, "out", 4)
+    _need(lse, torch.float32, "lse", 3)
     rc = load().gqa_splitkv_combine(_ptr(o_part), _ptr(lse_part), S, _ptr(sink), _ptr(out), _ptr(lse),
                                     B, Hq, Tq, d, _stream(stream))
     _check("gqa_splitkv_combine", rc)

@@ -282,15 +282,21 @@ int dispatch_fwd(const Params& p, const void* q, const void* k, const void* v, i
     }
 }
 
-long long timeout_cycles(const DeviceState& s) {
-    // about one second of SM clock, overridable for tests (GQA_WAIT_TIMEOUT_MS)
+// About one second of SM clock for every wait inside the kernels; tests shorten
+// it with GQA_WAIT_TIMEOUT_US (microseconds) or GQA_WAIT_TIMEOUT_MS.
+long long wait_limit_cycles(long long clock_khz) {
+    if (const char* e = std::getenv("GQA_WAIT_TIMEOUT_US")) {
+        const long long us = std::atoll(e);
+        if (us > 0) return clock_khz * us / 1000;
+    }
     long long ms = 1000;
     if (const char* e = std::getenv("GQA_WAIT_TIMEOUT_MS")) {
-        long long v = std::atoll(e);
+        const long long v = std::atoll(e);
         if (v > 0) ms = v;
     }
-    return s.clock_khz * ms;
+    return clock_khz * ms;
 }
+long long timeout_cycles(const DeviceState& s) { return wait_limit_cycles(s.clock_khz); }
 
 int ensure_counters(DeviceState& s, long long n) {
     if (s.counters_len >= n) return GQA_OK;
@@ -558,23 +564,6 @@ extern "C" int gqa_profile_take(float* kernel_ms, int max_calls, int* n_calls) {
     return GQA_OK;
 }
 
-extern "C" int gqa_get_device_error(gqa_stream_t stream) {
-    std::lock_guard<std::mutex> lk(g_mu);
-    DeviceState* s = nullptr;
-    int rc = get_state(&s);
-    if (rc) return rc;
-    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return GQA_ERR_CUDA;
-    int v = 0;
-    if (cudaMemcpy(&v, s->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GQA_ERR_CUDA;
-    if (v != 0) {
-        if (cudaMemset(s->err, 0, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
-        // an aborted launch may leave merge tickets behind
-        if (s->counters && cudaMemset(s->counters, 0, sizeof(int) * static_cast<size_t>(s->counters_len)) != cudaSuccess)
-            return GQA_ERR_CUDA;
-    }
-    return v;
-}
-
 extern "C" const char* gqa_status_string(int status) {
     switch (status) {
         case GQA_OK: return "ok";
@@ -587,6 +576,7 @@ extern "C" const char* gqa_status_string(int status) {
         case GQA_ERR_UNSUPPORTED: return "unsupported head dim or GPU";
         case GQA_ERR_KVLEN: return "a kv_lens value was outside [0, Tkv] and was clamped";
         case GQA_ERR_PAGE: return "a page id was outside [0, num_pages); page 0 was read instead";
+        case GQA_ERR_SMEM_ALIGN: return "a kernel's dynamic shared memory was not 1024-byte aligned (internal error)";
         case GQA_ERR_SCRATCH:
             return "the problem needs more scratch than is in place (the allocation-free array, or a call being "
                    "captured into a CUDA graph before an uncaptured call of that size)";
@@ -681,12 +671,7 @@ extern "C" int gqa_attention_fwd_noalloc(const void* q, const void* k, const voi
     if (rc) return rc;
     if (s->cc_major != 10) return GQA_ERR_UNSUPPORTED;
     Params p;
-    long long ms = 1000;
-    if (const char* e = std::getenv("GQA_WAIT_TIMEOUT_MS")) {
-        const long long v2 = std::atoll(e);
-        if (v2 > 0) ms = v2;
-    }
-    fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale, causal, kv_lens, sink, out, lse, 0, s->clock_khz * ms);
+    fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale, causal, kv_lens, sink, out, lse, 0, wait_limit_cycles(s->clock_khz));
     choose_geometry(p);
     if (p.W > static_cast<long long>(kNaCounterInts)) return GQA_ERR_SCRATCH;
     // as many CTAs (one per SM) as the fixed partial area can give two slots each
@@ -719,3 +704,43 @@ extern "C" int gqa_attention_fwd_noalloc(const void* q, const void* k, const voi
     if (uses_combine_kernel(d)) return launch_streamk_combine(p, 1, s->sm_count, st);
     return GQA_OK;
 }
+
+// Reads (and clears) the device error words of the current device: the
+// allocating entry points' word (only if they have run here: reading it never
+// allocates) and the fixed array's word of the allocation-free entry point
+// (only if it has run here).  The first non-zero word is returned.
+extern "C" int gqa_get_device_error(gqa_stream_t stream) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GQA_ERR_CUDA;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return GQA_ERR_CUDA;
+    int first = 0;
+    DeviceState& s = g_dev[dev];
+    if (s.init) {
+        int v = 0;
+        if (cudaMemcpy(&v, s.err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GQA_ERR_CUDA;
+        if (v != 0) {
+            if (cudaMemset(s.err, 0, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
+            // an aborted launch may leave merge tickets behind
+            if (s.counters && cudaMemset(s.counters, 0, sizeof(int) * static_cast<size_t>(s.counters_len)) != cudaSuccess)
+                return GQA_ERR_CUDA;
+            first = v;
+        }
+    }
+    const NoAllocDevice& na = g_na_dev[dev];
+    if (na.ready) {
+        int v = 0;
+        if (cudaMemcpy(&v, na.scratch + kNaErrOffset, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+            return GQA_ERR_CUDA;
+        if (v != 0) {
+            // the error word, the combine-job counters and the merge tickets (each
+            // call clears the tickets it uses, but an aborted launch may leave
+            // others behind)
+            if (cudaMemset(na.scratch + kNaErrOffset, 0, 32) != cudaSuccess) return GQA_ERR_CUDA;
+            if (cudaMemset(na.scratch, 0, kNaCounterInts * sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
+            if (first == 0) first = v;
+        }
+    }
+    return first;
+}
+

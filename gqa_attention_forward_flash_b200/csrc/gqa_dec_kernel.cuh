@@ -164,7 +164,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint8_t* smem = smem_raw;
     const uint32_t sbase = ptx::smem_addr(smem);
     if (sbase & 1023u) {  // the swizzled tiles need a 1024-aligned window
-        if (threadIdx.x == 0) atomicCAS(p.err, 0, DEV_ERR_TIMEOUT);
+        if (threadIdx.x == 0) atomicCAS(p.err, 0, DEV_ERR_SMEM_ALIGN);
         return;
     }
     const uint32_t bar0 = sbase + C::OFF_BAR;

@@ -58,6 +58,7 @@ constexpr int kMaxCombinePieces = 512;  // CTA groups of a split (the grid is at
 constexpr int DEV_ERR_TIMEOUT = -6;
 constexpr int DEV_ERR_KVLEN = -8;
 constexpr int DEV_ERR_PAGE = -10;
+constexpr int DEV_ERR_SMEM_ALIGN = -11;  // the dynamic shared-memory window was not 1024-byte aligned
 
 // A split row-block (one DSPLIT part of its O columns) whose pieces are all
 // written: the stream-K combine kernel merges it.

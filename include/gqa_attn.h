@@ -76,7 +76,9 @@ typedef enum {
     GQA_ERR_UNSUPPORTED = -7, /* head dim not in {64,128,256,512}, or the GPU is not sm_100 */
     GQA_ERR_KVLEN = -8,       /* a kv_lens value was outside [0, Tkv] (device-reported, clamped) */
     GQA_ERR_SCRATCH = -9,     /* the problem exceeds the scratch in place (noalloc's fixed array; graph capture) */
-    GQA_ERR_PAGE = -10        /* gqa_attention_fwd_paged: a page id outside [0, num_pages) (device-reported) */
+    GQA_ERR_PAGE = -10,       /* gqa_attention_fwd_paged: a page id outside [0, num_pages) (device-reported) */
+    GQA_ERR_SMEM_ALIGN = -11  /* a kernel's dynamic shared memory was not 1024-byte aligned; it computed
+                                 nothing (device-reported; an internal error, not an argument error) */
 } gqa_status;
 
 #define GQA_MAX_SPLITS 256
@@ -193,21 +195,24 @@ int gqa_attention_fwd_paged(const void *q, const void *k_cache, const void *v_ca
  *
  * Same arguments, result and validation as gqa_attention_fwd.  The split
  * partials that gqa_attention_fwd keeps in a cudaMalloc'd buffer live here in
- * one fixed array inside the library (about 21.3 MiB: 20 MiB of fp32 partial
- * rows, their lse values, 65536 merge tickets and an error word), held by every
- * GPU that loads the library until the process exits.  Limits: at most 65536
- * row-blocks (a row-block is 128 packed query rows of one KV head, 256 when a KV
- * head has more than 128 packed rows), else GQA_ERR_SCRATCH; the grid uses at
- * most as many CTAs as the array has two partial slots for, which for head
- * dim 128 with more than 128 packed rows per KV head is fewer than the SM count.
+ * one fixed array inside the library (about 23.3 MiB: 20 MiB of fp32 partial
+ * rows, their lse values, 65536 merge tickets, an error word, the combine-job
+ * counters and a combine-job list of 65536 entries), held by every GPU that
+ * loads the library until the process exits.  Limits: at most 65536 row-blocks
+ * (a row-block is 128 packed query rows of one KV head, 256 when a KV head has
+ * more than 128 packed rows), else GQA_ERR_SCRATCH; d = 512 is not served
+ * (GQA_ERR_UNSUPPORTED); the grid uses at most as many CTAs as the array has two
+ * partial slots for: 80 for head dim 256 and for head dim 128 with more than 128
+ * packed rows per KV head, one per SM otherwise.
  * The first call on a device looks up the array's device address and the SM
  * count (no allocation); make that first call outside any stream capture.
  * Every call on a device shares the array and leaves its contents behind: each
- * call clears, on its stream, the tickets and the error word it uses, and calls
- * whose executions overlap on the GPU (on streams the caller does not order)
- * race on it.  Device-side errors (an expired bounded
- * wait, a clamped kv_lens value) are recorded in the array's error word and not
- * reported; diagnose with gqa_attention_fwd and gqa_get_device_error.
+ * call clears, on its stream, the tickets, the error word and the combine-job
+ * counters it uses, and calls whose executions overlap on the GPU (on streams
+ * the caller does not order) race on it.  Device-side errors (an expired bounded
+ * wait, a clamped kv_lens value) are recorded in the array's error word;
+ * gqa_get_device_error reads and clears it (without allocating) until the next
+ * call clears it.
  */
 int gqa_attention_fwd_noalloc(const void *q, const void *k, const void *v, const int32_t *kv_lens,
                               const float *sink, void *out, float *lse, int B, int Hq, int Hkv,
@@ -216,8 +221,11 @@ int gqa_attention_fwd_noalloc(const void *q, const void *k, const void *v, const
 /*
  * Waits for `stream`, then returns (and clears) the first error a kernel of
  * this library recorded on the current device since the last call: GQA_OK,
- * GQA_ERR_TIMEOUT or GQA_ERR_KVLEN; GQA_ERR_CUDA if the synchronisation itself
- * failed.
+ * GQA_ERR_TIMEOUT, GQA_ERR_KVLEN, GQA_ERR_PAGE or GQA_ERR_SMEM_ALIGN;
+ * GQA_ERR_CUDA if the synchronisation itself failed.  It reads the error word
+ * of the allocating entry points and that of gqa_attention_fwd_noalloc's fixed
+ * array, each only if its entry points have run on the device, and allocates
+ * nothing.
  */
 int gqa_get_device_error(gqa_stream_t stream);
 

@@ -134,3 +134,28 @@ def test_shard_entry_points_reject_bad_arguments_on_the_host(lib):
     assert c(P(16), rows_d + 2, P(16), 8, 2, None, P(16), P(16), 1, 4, 2, 64, None) == -3  # stride not 8-byte
     assert c(P(24), rows_d, P(16), 8, 2, None, P(16), P(16), 1, 4, 2, 64, None) == -3      # base misaligned
     assert c(None, rows_d, P(16), 8, 2, None, P(16), P(16), 1, 4, 2, 64, None) == -1
+
+
+def test_binding_wrappers_validate_before_calling(lib):
+    """Every wrapper checks dtype, rank, contiguity and device before the C call
+    (a wrong tensor never reaches a kernel); CPU tensors are refused here."""
+    import torch
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    q = torch.zeros((1, 4, 2, 64), dtype=bf)
+    k = torch.zeros((1, 1, 8, 64), dtype=bf)
+    op = torch.zeros((1, 4, 2, 3, 64), dtype=f32)
+    lp = torch.zeros((1, 4, 2, 3), dtype=f32)
+    with pytest.raises(ValueError):
+        binding.gqa_attention_fwd_partial(q, k, k, num_splits=3)
+    with pytest.raises(ValueError):
+        binding.gqa_attention_fwd_partial(q.float(), k, k, num_splits=3)
+    with pytest.raises(ValueError):
+        binding.gqa_splitkv_combine(op, lp)
+    with pytest.raises(ValueError):
+        binding.gqa_splitkv_combine(op.double(), lp)
+    with pytest.raises(ValueError):
+        binding.gqa_splitkv_combine(op.transpose(3, 4), lp)
+    with pytest.raises(ValueError):
+        binding.gqa_attention_fwd_noalloc(q, k, k)
+    with pytest.raises(ValueError):
+        binding.gqa_attention_fwd(q, k, k, kv_lens=torch.zeros(1, dtype=i32))

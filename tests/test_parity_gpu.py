@@ -37,6 +37,9 @@ SMALL = {
     "noncausal_prefill_d128": Workload("nc", B=1, Hq=8, Hkv=1, Tq=130, Tkv=515, d=128, seed=12),
     "d512_sink_nan": shrink(W["wide_head_sink_decode"], B=2, Tkv=700, kv_len=631),
     "d512_mha_noncausal": Workload("d512", B=1, Hq=2, Hkv=2, Tq=70, Tkv=200, d=512, seed=20),
+    # the wide-head workload's "N(0, 0.5)" read as variance 0.5 (sigma = sqrt(0.5)): the second reading
+    "d512_sink_nan_var_half": shrink(W["wide_head_sink_decode"], B=2, Tkv=700, kv_len=631,
+                                     sigma=math.sqrt(0.5)),
 }
 
 
@@ -166,9 +169,15 @@ def test_combine_kernel_on_oracle_partials():
 FULL = ["batched_decode", "short_q_long_kv", "full_causal_prefill", "wide_head_sink_decode"]
 
 
-@pytest.mark.parametrize("name", FULL)
+FULL_VARIANTS = {
+    # "N(0, 0.5)" read as variance 0.5 rather than standard deviation 0.5
+    "wide_head_sink_decode_var_half": shrink(W["wide_head_sink_decode"], sigma=math.sqrt(0.5)),
+}
+
+
+@pytest.mark.parametrize("name", FULL + sorted(FULL_VARIANTS))
 def test_parity_full_size_sampled(name):
-    w = W[name]
+    w = W[name] if name in W else FULL_VARIANTS[name]
     inp = make_inputs(w)
     o, l = run_gpu(inp)
     assert np.all(np.isfinite(o))
