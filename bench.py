@@ -523,18 +523,17 @@ def run_e2e(args, w, inp, dev, stream, nbytes, nflops, ws):
 
 
 def main_kernel_name(w: Workload) -> str:
-    """The kernel(s) gqa_attention_fwd launches for these sizes: the swap-AB decode
+    """The kernel gqa_attention_fwd launches for these sizes: the swap-AB decode
     kernel for head dim 128 with at most 16 packed rows per KV head, the two-lane
-    kernel for the other head dims 64/128, the single-lane kernel and the combine
-    kernel for 256/512."""
+    kernel for the other head dims 64/128, the wide kernel for 256/512."""
     if w.d == 128 and w.G * w.Tq <= 16:
         return "gqa_dec_kernel"
-    return "gqa_fwd2_kernel" if w.d <= 128 else "gqa_fwd_kernel + gqa_combine_streamk_kernel"
+    return "gqa_fwd2_kernel" if w.d <= 128 else "gqa_wide_kernel"
 
 
 def launches_per_call(w: Workload) -> int:
-    """Head dims 64/128 merge split rows inside the one kernel; 256/512 add the combine kernel."""
-    return 1 if w.d <= 128 else 2
+    """Every kernel merges its split rows inside itself: one launch per call."""
+    return 1
 
 
 def kernel_source_digest() -> str:

@@ -17,6 +17,7 @@
 
 #include "gqa_attn.h"
 #include "gqa_dec_kernel.cuh"
+#include "gqa_wide_kernel.cuh"
 
 namespace gqa {
 namespace {
@@ -159,42 +160,26 @@ using CDec16 = DecCfg<16>;
 using CDec8_P = DecCfg<8, true>;
 using CDec16_P = DecCfg<16, true>;
 bool uses_decode_kernel(const Params& p) { return p.d == 128 && p.mode == 0 && p.R <= DEC_NQ; }
-using Cfg256 = FwdCfg<256, 64, 3, 2, 1>;
-// Head dim 512: O (128 x 512 fp32) fills a whole TMEM, so O's columns are split
-// over a pair of CTAs (DSPLIT = 2) that each compute the full S.
-using Cfg512 = FwdCfg<512, 32, 2, 2, 1, 2>;
+// Head dims 256 and 512: the wide kernel (128-key tiles streamed in 64-column
+// chunks past a resident Q tile, in-kernel merge of split row-blocks).  At 512 a
+// 128 x 512 fp32 O fills a whole TMEM, so O's columns are split over a pair of
+// CTAs (DSPLIT = 2) that each compute the full S.
+using CW256 = WideCfg<256, 1>;
+using CW512 = WideCfg<512, 2>;
 
-int dsplit_for(int d) { return d == 512 ? Cfg512::DSPLIT : 1; }
-
-// Head dims served by the single-lane kernel merge their split row-blocks in a
-// second kernel spread over every SM (their partial rows are long: 256 or 512
-// columns, up to one piece per CTA group); the two-lane kernel merges in place.
-bool uses_combine_kernel(int d) { return d == 256 || d == 512; }
-
-int launch_streamk_combine(const Params& p, int ds, int sm_count, cudaStream_t st) {
-    gqa_combine_streamk_kernel<<<2 * sm_count, 256, 0, st>>>(p, ds, BM * p.RBQ);
-    return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
-}
+int dsplit_for(int d) { return d == 512 ? CW512::DSPLIT : 1; }
 
 // Tile geometry of the kernel that will serve these sizes.
 void choose_geometry(Params& p) {
-    if (p.d == 512) {
-        p.BN = Cfg512::BN;
-        p.RBQ = 1;
-    } else if (p.d == 256) {
-        p.BN = Cfg256::BN;
-        p.RBQ = 1;
-    } else {
-        p.BN = 128;
-        p.RBQ = (p.R <= BM) ? 1 : 2;
-    }
+    p.BN = 128;
+    p.RBQ = (p.d <= 128 && p.R > BM) ? 2 : 1;
     p.QW = (p.QT + p.RBQ - 1) / p.RBQ;
     p.W = static_cast<long long>(p.U) * p.QW;
 }
 
-// Kernel families: the single-lane kernel (head dims 256, 512), the two-lane
-// kernel (64, 128) and the swap-AB decode kernel (128, at most 16 packed rows).
-enum KernelKind { kSingleLane = 0, kTwoLane = 1, kDecode = 2 };
+// Kernel families: the wide kernel (head dims 256, 512), the two-lane kernel
+// (64, 128) and the swap-AB decode kernel (128, at most 16 packed rows).
+enum KernelKind { kWide = 0, kTwoLane = 1, kDecode = 2 };
 
 template <class C, int KIND>
 int launch_fwd(const Params& p0, const void* q, const void* k, const void* v, int grid, cudaStream_t stream,
@@ -209,7 +194,7 @@ int launch_fwd(const Params& p0, const void* q, const void* k, const void* v, in
         else if constexpr (KIND == kDecode)
             e = cudaFuncSetAttribute(gqa_dec_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         else
-            e = cudaFuncSetAttribute(gqa_fwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+            e = cudaFuncSetAttribute(gqa_wide_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return GQA_ERR_CUDA;
         attr_done[dev] = true;
     }
@@ -226,7 +211,7 @@ int launch_fwd(const Params& p0, const void* q, const void* k, const void* v, in
     const uint64_t kvcols = static_cast<uint64_t>(C::D);
     // few packed rows (decode): spread them over the four TMEM lane quadrants so
     // that every SM sub-partition takes a share of the softmax
-    p.spread = (KIND != kDecode && p.QT == 1 && p.R <= 96) ? 1 : 0;
+    p.spread = (KIND == kTwoLane && p.QT == 1 && p.R <= 96) ? 1 : 0;
     p.rq = (p.R + 3) / 4;
     if constexpr (KIND == kDecode)  // the 16-row Q tile of the transposed MMAs
         p.q_box_rows = qrows < static_cast<uint64_t>(DEC_NQ) ? static_cast<int>(qrows) : DEC_NQ;
@@ -247,8 +232,22 @@ int launch_fwd(const Params& p0, const void* q, const void* k, const void* v, in
         gqa_fwd2_kernel<C><<<grid, NUM_THREADS2, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     else if constexpr (KIND == kDecode)
         gqa_dec_kernel<C><<<grid, NUM_THREADS_DEC, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
-    else
-        gqa_fwd_kernel<C><<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    else {
+        // the stream-K merge waits for pieces written by other CTAs of the grid:
+        // every CTA must be resident at once, which a cooperative launch guarantees
+        // (or refuses); the uniform splits of mode 1 never wait on another CTA
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(grid));
+        cfg.blockDim = dim3(NUM_THREADS_W);
+        cfg.dynamicSmemBytes = C::SMEM_BYTES;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = (p.mode == 0) ? 1 : 0;
+        if (cudaLaunchKernelEx(&cfg, gqa_wide_kernel<C>, tq, tk, tv, p) != cudaSuccess) return GQA_ERR_CUDA;
+    }
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
     if (ev_after && cudaEventRecord(ev_after, stream) != cudaSuccess) return GQA_ERR_CUDA;
     return GQA_OK;
@@ -276,8 +275,8 @@ int dispatch_fwd(const Params& p, const void* q, const void* k, const void* v, i
                                   : launch_fwd<C2_128_DQ_P, kTwoLane>(p, q, k, v, grid, stream, e0, e1);
             return p.RBQ == 1 ? launch_fwd<C2_128_SK, kTwoLane>(p, q, k, v, grid, stream, e0, e1)
                               : launch_fwd<C2_128_DQ, kTwoLane>(p, q, k, v, grid, stream, e0, e1);
-        case 256: return launch_fwd<Cfg256, kSingleLane>(p, q, k, v, grid, stream, e0, e1);
-        case 512: return launch_fwd<Cfg512, kSingleLane>(p, q, k, v, grid, stream, e0, e1);
+        case 256: return launch_fwd<CW256, kWide>(p, q, k, v, grid, stream, e0, e1);
+        case 512: return launch_fwd<CW512, kWide>(p, q, k, v, grid, stream, e0, e1);
         default: return GQA_ERR_UNSUPPORTED;
     }
 }
@@ -349,26 +348,26 @@ int run_streamk(Params& p, const void* q, const void* k, const void* v, DeviceSt
     const size_t slot_rows = static_cast<size_t>(2 * NC) * ds * BM * p.RBQ;
     const size_t slot_o = slot_rows * (d / ds) * sizeof(float);
     const size_t slot_l = (slot_rows * sizeof(float) + 255) & ~static_cast<size_t>(255);
-    const size_t jobs = static_cast<size_t>(p.W) * ds * sizeof(CJob);
+    // merge counters: one ticket per row-block (head dims <= 128), a published /
+    // merged pair per row-block and O part (256, 512)
+    const long long nctr = 2 * p.W * ds + 2;
     cudaStream_t st0 = reinterpret_cast<cudaStream_t>(stream);
-    if (s->scratch_bytes < slot_o + slot_l + jobs || s->counters_len < p.W * ds + 2) {
+    if (s->scratch_bytes < slot_o + slot_l || s->counters_len < nctr) {
         // growing the scratch allocates (and synchronises): not while the stream is
         // being captured into a CUDA graph
         cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
         if (cudaStreamIsCapturing(st0, &cs) != cudaSuccess) return GQA_ERR_CUDA;
         if (cs != cudaStreamCaptureStatusNone) return GQA_ERR_SCRATCH;
     }
-    rc = ensure_scratch(*s, slot_o + slot_l + jobs);
+    rc = ensure_scratch(*s, slot_o + slot_l);
     if (rc) return rc;
-    rc = ensure_counters(*s, p.W * ds + 2);
+    rc = ensure_counters(*s, nctr);
     if (rc) return rc;
     char* base = static_cast<char*>(s->scratch);
     p.mode = 0;
     p.part_o = reinterpret_cast<float*>(base);
     p.part_lse = reinterpret_cast<float*>(base + slot_o);
-    p.cjobs = reinterpret_cast<CJob*>(base + slot_o + slot_l);
     p.counters = s->counters;
-    p.cjob_count = s->counters + p.W * ds;
     p.err = s->err;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaEvent_t* ev = nullptr;
@@ -377,14 +376,8 @@ int run_streamk(Params& p, const void* q, const void* k, const void* v, DeviceSt
         cudaGetDevice(&dev);
         if (dev == g_prof.dev) ev = g_prof.ev[g_prof.n++];
     }
-    const bool combine = uses_combine_kernel(d);
-    rc = dispatch_fwd(p, q, k, v, NC * ds, st, ev ? ev[0] : nullptr, (ev && !combine) ? ev[1] : nullptr);
+    rc = dispatch_fwd(p, q, k, v, NC * ds, st, ev ? ev[0] : nullptr, ev ? ev[1] : nullptr);
     if (rc) return rc;
-    if (combine) {
-        rc = launch_streamk_combine(p, ds, s->sm_count, st);
-        if (rc) return rc;
-        if (ev && cudaEventRecord(ev[1], st) != cudaSuccess) return GQA_ERR_CUDA;
-    }
     return GQA_OK;
 }
 
@@ -600,15 +593,13 @@ extern "C" int gqa_version(void) { return 100; }
 namespace gqa {
 namespace {
 
-constexpr size_t kNaCounterInts = 65536;                         // merge tickets: at most this many row-blocks
+constexpr size_t kNaCounterInts = 65536;                         // merge counters
 constexpr size_t kNaErrOffset = kNaCounterInts * sizeof(int);    // device error word
-constexpr size_t kNaJobCountOffset = kNaErrOffset + 16;           // combine jobs listed / blocks done
 constexpr size_t kNaLseOffset = kNaErrOffset + 256;
 constexpr size_t kNaLseFloats = static_cast<size_t>(2) * kMaxCtas * 2 * BM;  // 2 slots x 256 rows per CTA
 constexpr size_t kNaPartOffset = kNaLseOffset + kNaLseFloats * sizeof(float);
 constexpr size_t kNaPartBytes = static_cast<size_t>(20) << 20;  // fp32 partial O: 20 MiB
-constexpr size_t kNaJobsOffset = kNaPartOffset + kNaPartBytes;  // combine jobs: one per row-block at most
-constexpr size_t kNaBytes = kNaJobsOffset + kNaCounterInts * sizeof(CJob);  // about 23.3 MiB in all
+constexpr size_t kNaBytes = kNaPartOffset + kNaPartBytes;       // about 21.3 MiB in all
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNaBytes];
 
@@ -664,7 +655,6 @@ extern "C" int gqa_attention_fwd_noalloc(const void* q, const void* k, const voi
     if (B == 0 || Tq == 0) return GQA_OK;
     if (!out) return GQA_ERR_NULL;
     if (!aligned16(out) || (lse && !aligned16(lse))) return GQA_ERR_ALIGN;
-    if (d == 512) return GQA_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lk(g_mu);
     NoAllocDevice* s = nullptr;
     rc = noalloc_setup(&s);
@@ -673,12 +663,16 @@ extern "C" int gqa_attention_fwd_noalloc(const void* q, const void* k, const voi
     Params p;
     fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale, causal, kv_lens, sink, out, lse, 0, wait_limit_cycles(s->clock_khz));
     choose_geometry(p);
-    if (p.W > static_cast<long long>(kNaCounterInts)) return GQA_ERR_SCRATCH;
-    // as many CTAs (one per SM) as the fixed partial area can give two slots each
+    const int ds = dsplit_for(d);
+    // merge counters: a ticket per row-block (head dims <= 128), a published /
+    // merged pair per row-block and O part (256, 512)
+    const long long nctr = (d >= 256) ? 2 * p.W * ds : p.W;
+    if (nctr > static_cast<long long>(kNaCounterInts)) return GQA_ERR_SCRATCH;
+    // as many CTA groups (one CTA per SM) as the fixed partial area can give two slots each
     const size_t rows_per_slot = static_cast<size_t>(BM) * p.RBQ;
-    const size_t per_cta = 2 * rows_per_slot * static_cast<size_t>(d) * sizeof(float);
-    long long NC = s->sm_count < kMaxCtas ? s->sm_count : kMaxCtas;
-    if (static_cast<long long>(kNaPartBytes / per_cta) < NC) NC = static_cast<long long>(kNaPartBytes / per_cta);
+    const size_t per_group = 2 * rows_per_slot * static_cast<size_t>(d) * sizeof(float);
+    long long NC = (s->sm_count < kMaxCtas ? s->sm_count : kMaxCtas) / ds;
+    if (static_cast<long long>(kNaPartBytes / per_group) < NC) NC = static_cast<long long>(kNaPartBytes / per_group);
     if (!kv_lens) {
         long long tot = 0;
         for (int qw = 0; qw < p.QW; ++qw) tot += qtile_ntiles(p, qw, Tkv);
@@ -692,16 +686,13 @@ extern "C" int gqa_attention_fwd_noalloc(const void* q, const void* k, const voi
     p.part_lse = reinterpret_cast<float*>(base + kNaLseOffset);
     p.counters = reinterpret_cast<int*>(base);
     p.err = reinterpret_cast<int*>(base + kNaErrOffset);
-    p.cjobs = reinterpret_cast<CJob*>(base + kNaJobsOffset);
-    p.cjob_count = reinterpret_cast<int*>(base + kNaJobCountOffset);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // the array keeps the last call's contents: the merge tickets, the error word
-    // and the combine-job counters must start at zero
-    if (cudaMemsetAsync(base, 0, static_cast<size_t>(p.W) * sizeof(int), st) != cudaSuccess) return GQA_ERR_CUDA;
+    // the array keeps the last call's contents: the merge counters and the error
+    // word must start at zero
+    if (cudaMemsetAsync(base, 0, static_cast<size_t>(nctr) * sizeof(int), st) != cudaSuccess) return GQA_ERR_CUDA;
     if (cudaMemsetAsync(base + kNaErrOffset, 0, 32, st) != cudaSuccess) return GQA_ERR_CUDA;
-    rc = dispatch_fwd(p, q, k, v, static_cast<int>(NC), st);
+    rc = dispatch_fwd(p, q, k, v, static_cast<int>(NC * ds), st);
     if (rc) return rc;
-    if (uses_combine_kernel(d)) return launch_streamk_combine(p, 1, s->sm_count, st);
     return GQA_OK;
 }
 

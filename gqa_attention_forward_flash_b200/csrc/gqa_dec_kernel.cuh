@@ -221,6 +221,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ptx::fence_proxy_async_smem();
     }
     ptx::tc_fence_before();
+    __syncwarp();
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = misc->tmem_base;
@@ -701,7 +702,12 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
 
     // ---------------------------------------------------------------- teardown
+    // A role ran in one lane of its warp while the other lanes went ahead: the
+    // warp reconverges first, so that the CTA barrier below counts every thread
+    // (a divergent warp at a CTA barrier can release it early, and TMEM would
+    // then be freed while the softmax warps still read it).
     ptx::tc_fence_before();
+    __syncwarp();
     __syncthreads();
     if (warp == 2) {
         ptx::tc_fence_after();

@@ -28,9 +28,9 @@
 // producer.  Each single-thread role has a warp of its own, so no role's spin
 // on a barrier delays another's issue.
 // Work split, logical-length masking, the sink, split partials and the
-// last-arriver merge follow the single-lane kernel (gqa_fwd_kernel.cuh).
+// last-arriver merge use the pieces in gqa_common.cuh.
 #pragma once
-#include "gqa_fwd_kernel.cuh"
+#include "gqa_common.cuh"
 
 namespace gqa {
 
@@ -212,6 +212,7 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     if (p.mode == 0 && warp == 8) plan_span(p, cta, NC, &misc->span);
     ptx::tc_fence_before();
+    __syncwarp();
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = misc->tmem_base;
@@ -839,7 +840,12 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
 
     // ---------------------------------------------------------------- teardown
+    // A role ran in one lane of its warp while the other lanes went ahead: the
+    // warp reconverges first, so that the CTA barrier below counts every thread
+    // (a divergent warp at a CTA barrier can release it early, and TMEM would
+    // then be freed while the softmax warps still read it).
     ptx::tc_fence_before();
+    __syncwarp();
     __syncthreads();
     if (warp == 9) {
         ptx::tc_fence_after();

@@ -195,20 +195,20 @@ int gqa_attention_fwd_paged(const void *q, const void *k_cache, const void *v_ca
  *
  * Same arguments, result and validation as gqa_attention_fwd.  The split
  * partials that gqa_attention_fwd keeps in a cudaMalloc'd buffer live here in
- * one fixed array inside the library (about 23.3 MiB: 20 MiB of fp32 partial
- * rows, their lse values, 65536 merge tickets, an error word, the combine-job
- * counters and a combine-job list of 65536 entries), held by every GPU that
- * loads the library until the process exits.  Limits: at most 65536 row-blocks
- * (a row-block is 128 packed query rows of one KV head, 256 when a KV head has
- * more than 128 packed rows), else GQA_ERR_SCRATCH; d = 512 is not served
- * (GQA_ERR_UNSUPPORTED); the grid uses at most as many CTAs as the array has two
- * partial slots for: 80 for head dim 256 and for head dim 128 with more than 128
- * packed rows per KV head, one per SM otherwise.
+ * one fixed array inside the library (about 21.3 MiB: 20 MiB of fp32 partial
+ * rows, their lse values, 65536 merge counters and an error word), held by
+ * every GPU that loads the library until the process exits.  Limits: the merge
+ * counters cover at most 65536 row-blocks for head dims 64 and 128, 32768 for
+ * 256 and 16384 for 512 (a row-block is 128 packed query rows of one KV head,
+ * 256 when a KV head has more than 128 packed rows at head dim 64 or 128), else
+ * GQA_ERR_SCRATCH; the grid uses at most as many CTAs as the array has two
+ * partial slots for: 80 for head dims 256 and 512 and for head dim 128 with
+ * more than 128 packed rows per KV head, one per SM otherwise.
  * The first call on a device looks up the array's device address and the SM
  * count (no allocation); make that first call outside any stream capture.
  * Every call on a device shares the array and leaves its contents behind: each
- * call clears, on its stream, the tickets, the error word and the combine-job
- * counters it uses, and calls whose executions overlap on the GPU (on streams
+ * call clears, on its stream, the merge counters and the error word it uses,
+ * and calls whose executions overlap on the GPU (on streams
  * the caller does not order) race on it.  Device-side errors (an expired bounded
  * wait, a clamped kv_lens value) are recorded in the array's error word;
  * gqa_get_device_error reads and clears it (without allocating) until the next
@@ -233,7 +233,8 @@ int gqa_get_device_error(gqa_stream_t stream);
  * Measurement hook (no counterpart on the pages; it only observes).  After
  * gqa_profile_begin, each gqa_attention_fwd call on the current device (up to
  * 4096 calls) records CUDA events on its own stream right before and right
- * after its kernel (one launch per call: the split-KV merge runs inside it).
+ * after its kernel (one launch per call: the split-KV merge runs inside it,
+ * for every head dim).
  * gqa_profile_take stops recording, waits for those events and writes, per
  * call, the kernel's duration in ms into kernel_ms[0 .. *n_calls) (kernel_ms
  * may be NULL; at most max_calls entries).

@@ -1,7 +1,7 @@
 """CUDA graphs: calls into the library captured in a graph and replayed give the
 eager results bit for bit (the kernels are deterministic and take every size
 through kernel parameters), for the swap-AB decode kernel, the two-lane kernel
-and the single-lane kernel with its combine launch; a captured call that would
+and the wide kernel (cooperative launch, in-kernel merge); a captured call that would
 need more scratch than is in place is refused, not allocated."""
 import pytest
 import torch
@@ -14,7 +14,7 @@ pytestmark = pytest.mark.gpu
 CASES = {
     "decode_swap_ab": shrink(WORKLOADS["batched_decode"], B=4, Tkv=3000),
     "prefill_two_lane": Workload("gp", B=1, Hq=8, Hkv=2, Tq=300, Tkv=700, d=128, causal=True, sink=True, seed=91),
-    "wide_single_lane": shrink(WORKLOADS["wide_head_sink_decode"], B=2, Tkv=1500, kv_len=1403),
+    "wide_head_d512": shrink(WORKLOADS["wide_head_sink_decode"], B=2, Tkv=1500, kv_len=1403),
 }
 
 

@@ -12,8 +12,8 @@ array must read back as zero through gqa_get_device_error.
 
 The cases cover the three kernel families: the swap-AB decode kernel (head
 dim 128, few packed rows), the two-lane kernel (head dims 64 and 128, split-key
-and dual-Q lanes) and the single-lane kernel with the stream-K combine kernel
-(head dim 256), whose job list also lives in the fixed array.
+and dual-Q lanes) and the wide kernel (head dims 256 and 512), whose merge
+counters also live in the fixed array.
 
 This file is named so that pytest collects it last: a run that stops at the
 first failure has then already run every other test.
@@ -37,10 +37,11 @@ CASES = {
     "causal_prefill": shrink(WORKLOADS["full_causal_prefill"], B=1, Hq=8, Hkv=2, Tq=1100, Tkv=1100),
     "d64_causal_sink": Workload("d64", B=2, Hq=8, Hkv=2, Tq=37, Tkv=900, d=64, causal=True, ragged=True,
                                 nan_pad=True, sink=True, seed=21),
-    # head dim 256: the single-lane kernel lists its split row-blocks in the
-    # array's job list and the combine kernel merges them
+    # head dims 256 and 512: the wide kernel's split row-blocks are merged in the
+    # kernel, with their counters in the array
     "d256_sink_nan_split": Workload("d256", B=2, Hq=16, Hkv=2, Tq=3, Tkv=6000, d=256, sigma=0.5, causal=True,
                                     sink=True, kv_len=5555, nan_pad=True, seed=22),
+    "d512_sink_nan_split": shrink(WORKLOADS["wide_head_sink_decode"], B=2, Tkv=3000, kv_len=2903),
 }
 
 
