@@ -14,7 +14,11 @@ Recipe (per workload below):
   * K and V rows at positions >= kv_len (the padded capacity) are overwritten
     with NaN where the workload asks for NaN padding, so that any read of a
     padded row shows up in the output;
-  * sink: ``randn`` float32 per query head (already in the scaled-logit domain).
+  * sink: ``randn`` float32 per query head (already in the scaled-logit domain);
+  * FP8 K/V (workloads with ``kv_fp8``): K and V drawn as above, then stored as
+    OCP FP8 E4M3 with one scale per tensor, the AstrAI fp8 quantize recipe:
+    scale = amax / 448 over the tensor's finite values, bytes = (x / scale)
+    rounded to E4M3 by torch's cast (the NaN padding stays NaN).
 
 The five named workloads are the shapes the pages measure or describe: the
 tiny prefill, the batched decode with ragged lengths, the short-query/long-KV
@@ -47,6 +51,7 @@ class Workload:
     ragged: bool = False        # kv_len ~ U[1, Tkv] per batch
     nan_pad: bool = False       # K/V rows >= kv_len are NaN
     seed: int = 0
+    kv_fp8: bool = False        # K/V stored as E4M3 bytes with per-tensor scales
 
     @property
     def G(self) -> int:
@@ -69,6 +74,9 @@ WORKLOADS = {
     "wide_head_sink_decode": Workload("wide_head_sink_decode", B=8, Hq=32, Hkv=1, Tq=4, Tkv=8192,
                                       d=512, sigma=0.5, causal=True, sink=True, kv_len=8131,
                                       nan_pad=True, seed=1005),
+    # the batched decode with its K/V cache in FP8 (E4M3, per-tensor scales)
+    "batched_decode_fp8kv": Workload("batched_decode_fp8kv", B=16, Hq=32, Hkv=4, Tq=1, Tkv=16384, d=128,
+                                     ragged=True, nan_pad=True, seed=1006, kv_fp8=True),
 }
 
 
@@ -86,6 +94,10 @@ class Inputs:
     sink: torch.Tensor | None      # float32 [Hq]
     scale: float
     causal: bool
+    k8: torch.Tensor | None = None   # E4M3 [B, Hkv, Tkv, d] (kv_fp8 workloads)
+    v8: torch.Tensor | None = None
+    k_scale: float = 1.0
+    v_scale: float = 1.0
 
 
 def make_inputs(w: Workload, seed: int | None = None) -> Inputs:
@@ -115,7 +127,24 @@ def make_inputs(w: Workload, seed: int | None = None) -> Inputs:
                 k[b, :, n:, :] = float("nan")
                 v[b, :, n:, :] = float("nan")
     sink = torch.randn((w.Hq,), generator=g, dtype=torch.float32) if w.sink else None
-    return Inputs(q=q, k=k, v=v, kv_lens=kv_lens, sink=sink, scale=w.scale, causal=w.causal)
+    inp = Inputs(q=q, k=k, v=v, kv_lens=kv_lens, sink=sink, scale=w.scale, causal=w.causal)
+    if w.kv_fp8:
+        inp.k8, inp.k_scale = to_e4m3(k)
+        inp.v8, inp.v_scale = to_e4m3(v)
+    return inp
+
+
+E4M3_MAX = 448.0
+
+
+def to_e4m3(x: torch.Tensor):
+    """One tensor as E4M3 bytes and its scale: scale = amax / 448 over the finite
+    values, bytes = x / scale rounded by torch's cast (NaN stays NaN)."""
+    xf = x.float()
+    fin = torch.isfinite(xf)
+    amax = float(xf[fin].abs().max()) if bool(fin.any()) else 1.0
+    scale = amax / E4M3_MAX if amax > 0 else 1.0
+    return (xf / scale).to(torch.float8_e4m3fn), scale
 
 
 

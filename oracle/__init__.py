@@ -16,6 +16,10 @@ Functions (each restates the definition written in the C file's header):
 * :func:`attention_rows` -- the full forward for a list of flat rows
   ``(b*Hq + h)*Tq + i`` only (for sampled checks at full size).
 * :func:`combine` -- the LSE merge of per-split partials.
+* :func:`attention_fp8kv`, :func:`attention_rows_fp8kv` -- the forward with K and
+  V stored as OCP FP8 E4M3 bytes and one scale per tensor (K = value(k) * k_scale,
+  V = value(v) * v_scale), computed in double.
+* :func:`e4m3_decode` -- the E4M3 byte decoder those use.
 """
 from __future__ import annotations
 
@@ -53,6 +57,12 @@ def _load():
         lib.oracle_attention_window.restype = I
         lib.oracle_attention_rows.argtypes = [P, P, P, P, P, P, L, P, P, I, I, I, I, I, I, D, I, I]
         lib.oracle_attention_rows.restype = I
+        lib.oracle_attention_window_fp8kv.argtypes = [P, P, P, D, D, P, P, P, P, I, I, I, I, I, I, D, I, L, L, I]
+        lib.oracle_attention_window_fp8kv.restype = I
+        lib.oracle_attention_rows_fp8kv.argtypes = [P, P, P, D, D, P, P, P, L, P, P, I, I, I, I, I, I, D, I, I]
+        lib.oracle_attention_rows_fp8kv.restype = I
+        lib.oracle_e4m3_decode.argtypes = [P, P, L]
+        lib.oracle_e4m3_decode.restype = None
         lib.oracle_combine.argtypes = [P, P, I, P, P, P, I, I, I, I]
         lib.oracle_combine.restype = I
         lib.oracle_num_threads.argtypes = []
@@ -162,4 +172,73 @@ def combine(o_part, lse_part, sink=None):
     if rc != 0:
         raise ValueError("oracle_combine failed: %d" % rc)
     del sk
+    return out, lse
+
+
+def _bytes(x) -> np.ndarray:
+    """E4M3 tensor/array (torch.float8_e4m3fn or uint8) -> contiguous uint8 bytes."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().contiguous()
+            if x.dtype != torch.uint8:
+                assert x.dtype == torch.float8_e4m3fn
+                x = x.view(torch.uint8)
+            return np.ascontiguousarray(x.numpy())
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.asarray(x)
+    assert a.dtype == np.uint8
+    return np.ascontiguousarray(a)
+
+
+def e4m3_decode(x) -> np.ndarray:
+    """Values (fp64) of E4M3 bytes."""
+    b = _bytes(x)
+    out = np.zeros(b.shape, np.float64)
+    _load().oracle_e4m3_decode(b.ctypes.data, out.ctypes.data, b.size)
+    return out
+
+
+def attention_fp8kv(q, k8, v8, k_scale, v_scale, kv_lens=None, sink=None, scale=None, causal=False, threads=0):
+    """The full forward on K = value(k8) * k_scale, V = value(v8) * v_scale.
+
+    q: bf16 [B, Hq, Tq, d]; k8, v8: E4M3 [B, Hkv, Tkv, d].  Returns (out fp64
+    [B,Hq,Tq,d], lse fp64 [B,Hq,Tq])."""
+    qb, kb, vb = _bits(q), _bytes(k8), _bytes(v8)
+    B, Hq, Tq, d = qb.shape
+    _, Hkv, Tkv, _ = kb.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    kl, klp = _opt(kv_lens, np.int32)
+    sk, skp = _opt(sink, np.float32)
+    out = np.zeros((B, Hq, Tq, d), np.float64)
+    lse = np.zeros((B, Hq, Tq), np.float64)
+    rc = _load().oracle_attention_window_fp8kv(
+        qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, float(k_scale), float(v_scale), klp, skp,
+        out.ctypes.data, lse.ctypes.data, B, Hq, Hkv, Tq, Tkv, d, float(scale), int(bool(causal)),
+        0, int(Tkv), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_attention_window_fp8kv failed: %d" % rc)
+    del kl, sk
+    return out, lse
+
+
+def attention_rows_fp8kv(q, k8, v8, k_scale, v_scale, kv_lens, sink, scale, causal, rows, threads=0):
+    """attention_fp8kv at flat rows ``(b*Hq + h)*Tq + i`` only: (out fp64 [n, d], lse fp64 [n])."""
+    qb, kb, vb = _bits(q), _bytes(k8), _bytes(v8)
+    B, Hq, Tq, d = qb.shape
+    _, Hkv, Tkv, _ = kb.shape
+    kl, klp = _opt(kv_lens, np.int32)
+    sk, skp = _opt(sink, np.float32)
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    out = np.zeros((r.size, d), np.float64)
+    lse = np.zeros((r.size,), np.float64)
+    rc = _load().oracle_attention_rows_fp8kv(
+        qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, float(k_scale), float(v_scale), klp, skp,
+        r.ctypes.data, r.size, out.ctypes.data, lse.ctypes.data, B, Hq, Hkv, Tq, Tkv, d, float(scale),
+        int(bool(causal)), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_attention_rows_fp8kv failed: %d" % rc)
+    del kl, sk
     return out, lse

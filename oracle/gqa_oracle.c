@@ -36,6 +36,17 @@
  * Layouts: q/out [B, Hq, Tq, d], k/v [B, Hkv, Tkv, d], lse [B, Hq, Tq], all
  * contiguous; Tkv is the buffer capacity.
  *
+ * FP8 K/V (the *_fp8kv entry points): K and V are stored as OCP FP8 E4M3 bytes
+ * with one scale per tensor, the format of the AstrAI commit log's fp8 family
+ * (e4m3 quantize with a per-tensor scale; the consumer multiplies back by the
+ * scale).  The value of a byte (sign s, exponent field e, mantissa field m,
+ * exponent bias 7):
+ *     e = 0            (-1)^s * 2^-6 * m/8          (subnormal)
+ *     e = 15, m = 7    NaN                          (the format has no infinities)
+ *     otherwise        (-1)^s * 2^(e-7) * (1 + m/8)
+ * and the attention above is computed on K = value(k) * k_scale and
+ * V = value(v) * v_scale, in double.
+ *
  * Every function here is pinned by the CPU tests (closed forms, invariants,
  * brute force at high precision), none by this code itself.
  */
@@ -54,9 +65,39 @@ static double bf16_bits_to_double(uint16_t h) {
     return (double)f;
 }
 
+/* OCP FP8 E4M3 byte -> double (the table in the header comment). */
+static double e4m3_to_double(uint8_t x) {
+    const int s = x >> 7, e = (x >> 3) & 15, m = x & 7;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else if (e == 15 && m == 7)
+        return NAN;
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* K and V elements: bf16 bit patterns (kv_fmt 0) or E4M3 bytes times a
+ * per-tensor scale (kv_fmt 1). */
+typedef struct {
+    const void *k, *v;
+    int fmt;
+    double k_scale, v_scale;
+} kv_src;
+
+static double kv_k(const kv_src *s, long idx) {
+    return s->fmt ? e4m3_to_double(((const uint8_t *)s->k)[idx]) * s->k_scale
+                  : bf16_bits_to_double(((const uint16_t *)s->k)[idx]);
+}
+static double kv_v(const kv_src *s, long idx) {
+    return s->fmt ? e4m3_to_double(((const uint8_t *)s->v)[idx]) * s->v_scale
+                  : bf16_bits_to_double(((const uint16_t *)s->v)[idx]);
+}
+
 /* One output row (b, h, i) over the visible keys restricted to [kv_begin, kv_end).
  * s_buf must hold at least Tkv doubles. */
-static void attend_row(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+static void attend_row(const uint16_t *q, const kv_src *kv,
                        const int32_t *kv_lens, const float *sink,
                        int B, int Hq, int Hkv, int Tq, int Tkv, int d,
                        double scale, int causal, long kv_begin, long kv_end,
@@ -75,14 +116,14 @@ static void attend_row(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     if (kv_end - 1 < last) last = kv_end - 1;
 
     const uint16_t *qr = q + (((long)b * Hq + h) * Tq + i) * (long)d;
-    const uint16_t *kb = k + ((long)b * Hkv + g) * (long)Tkv * d;
-    const uint16_t *vb = v + ((long)b * Hkv + g) * (long)Tkv * d;
+    const long kb = ((long)b * Hkv + g) * (long)Tkv * d;  /* first element of the head's K / V rows */
+    const long vb = kb;
 
     double M = -INFINITY;
     for (long j = first; j <= last; ++j) {
-        const uint16_t *kr = kb + j * (long)d;
+        const long kr = kb + j * (long)d;
         double acc = 0.0;
-        for (int c = 0; c < d; ++c) acc += bf16_bits_to_double(qr[c]) * bf16_bits_to_double(kr[c]);
+        for (int c = 0; c < d; ++c) acc += bf16_bits_to_double(qr[c]) * kv_k(kv, kr + c);
         double s = scale * acc;
         s_buf[j] = s;
         if (s > M) M = s;
@@ -100,8 +141,8 @@ static void attend_row(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     for (long j = first; j <= last; ++j) {
         double p = exp(s_buf[j] - M);
         Z += p;
-        const uint16_t *vr = vb + j * (long)d;
-        for (int c = 0; c < d; ++c) o_row[c] += p * bf16_bits_to_double(vr[c]);
+        const long vr = vb + j * (long)d;
+        for (int c = 0; c < d; ++c) o_row[c] += p * kv_v(kv, vr + c);
     }
     if (has_sink) Z += exp(sk - M);
     for (int c = 0; c < d; ++c) o_row[c] /= Z;
@@ -118,7 +159,7 @@ static int check_shape(int B, int Hq, int Hkv, int Tq, int Tkv, int d) {
  * visible set: the partial result of one split of the keys.  kv_begin = 0 and
  * kv_end >= Tkv gives the full attention.  out: double [B,Hq,Tq,d]; lse: double
  * [B,Hq,Tq].  nthreads <= 0 uses the OpenMP default. */
-int oracle_attention_window(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+static int attention_window(const uint16_t *q, const kv_src *kv,
                             const int32_t *kv_lens, const float *sink,
                             double *out, double *lse,
                             int B, int Hq, int Hkv, int Tq, int Tkv, int d,
@@ -145,13 +186,37 @@ int oracle_attention_window(const uint16_t *q, const uint16_t *k, const uint16_t
                 int i = (int)(r % Tq);
                 int h = (int)((r / Tq) % Hq);
                 int b = (int)(r / ((long)Tq * Hq));
-                attend_row(q, k, v, kv_lens, sink, B, Hq, Hkv, Tq, Tkv, d, scale, causal,
+                attend_row(q, kv, kv_lens, sink, B, Hq, Hkv, Tq, Tkv, d, scale, causal,
                            kv_begin, kv_end, b, h, i, out + r * d, lse + r, s_buf);
             }
             free(s_buf);
         }
     }
     return fail ? -7 : 0;
+}
+
+int oracle_attention_window(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                            const int32_t *kv_lens, const float *sink,
+                            double *out, double *lse,
+                            int B, int Hq, int Hkv, int Tq, int Tkv, int d,
+                            double scale, int causal, long kv_begin, long kv_end,
+                            int nthreads) {
+    const kv_src kv = {k, v, 0, 1.0, 1.0};
+    return attention_window(q, &kv, kv_lens, sink, out, lse, B, Hq, Hkv, Tq, Tkv, d, scale, causal,
+                            kv_begin, kv_end, nthreads);
+}
+
+/* The same with E4M3 K / V bytes and their per-tensor scales. */
+int oracle_attention_window_fp8kv(const uint16_t *q, const uint8_t *k, const uint8_t *v,
+                                  double k_scale, double v_scale,
+                                  const int32_t *kv_lens, const float *sink,
+                                  double *out, double *lse,
+                                  int B, int Hq, int Hkv, int Tq, int Tkv, int d,
+                                  double scale, int causal, long kv_begin, long kv_end,
+                                  int nthreads) {
+    const kv_src kv = {k, v, 1, k_scale, v_scale};
+    return attention_window(q, &kv, kv_lens, sink, out, lse, B, Hq, Hkv, Tq, Tkv, d, scale, causal,
+                            kv_begin, kv_end, nthreads);
 }
 
 /* The full attention. */
@@ -166,7 +231,7 @@ int oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
 
 /* The full attention for a list of rows only: rows[r] = (b*Hq + h)*Tq + i.
  * out: double [nrows, d]; lse: double [nrows]. */
-int oracle_attention_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+static int attention_rows(const uint16_t *q, const kv_src *kv,
                           const int32_t *kv_lens, const float *sink,
                           const int64_t *rows, long nrows, double *out, double *lse,
                           int B, int Hq, int Hkv, int Tq, int Tkv, int d,
@@ -195,13 +260,39 @@ int oracle_attention_rows(const uint16_t *q, const uint16_t *k, const uint16_t *
                 int i = (int)(fr % Tq);
                 int h = (int)((fr / Tq) % Hq);
                 int b = (int)(fr / ((long)Tq * Hq));
-                attend_row(q, k, v, kv_lens, sink, B, Hq, Hkv, Tq, Tkv, d, scale, causal,
+                attend_row(q, kv, kv_lens, sink, B, Hq, Hkv, Tq, Tkv, d, scale, causal,
                            0, (long)Tkv, b, h, i, out + r * d, lse + r, s_buf);
             }
             free(s_buf);
         }
     }
     return fail ? -7 : 0;
+}
+
+int oracle_attention_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                          const int32_t *kv_lens, const float *sink,
+                          const int64_t *rows, long nrows, double *out, double *lse,
+                          int B, int Hq, int Hkv, int Tq, int Tkv, int d,
+                          double scale, int causal, int nthreads) {
+    const kv_src kv = {k, v, 0, 1.0, 1.0};
+    return attention_rows(q, &kv, kv_lens, sink, rows, nrows, out, lse, B, Hq, Hkv, Tq, Tkv, d,
+                          scale, causal, nthreads);
+}
+
+int oracle_attention_rows_fp8kv(const uint16_t *q, const uint8_t *k, const uint8_t *v,
+                                double k_scale, double v_scale,
+                                const int32_t *kv_lens, const float *sink,
+                                const int64_t *rows, long nrows, double *out, double *lse,
+                                int B, int Hq, int Hkv, int Tq, int Tkv, int d,
+                                double scale, int causal, int nthreads) {
+    const kv_src kv = {k, v, 1, k_scale, v_scale};
+    return attention_rows(q, &kv, kv_lens, sink, rows, nrows, out, lse, B, Hq, Hkv, Tq, Tkv, d,
+                          scale, causal, nthreads);
+}
+
+/* E4M3 bytes -> doubles (for the pins of the decoder). */
+void oracle_e4m3_decode(const uint8_t *in, double *out, long n) {
+    for (long i = 0; i < n; ++i) out[i] = e4m3_to_double(in[i]);
 }
 
 /* Merge S partial results per row.  o_part: float [rows, S, d] (each partial

@@ -385,8 +385,15 @@ MUTATIONS = {
     "double_normalisation": ("for (int c = 0; c < d; ++c) o_row[c] /= Z;",
                              "for (int c = 0; c < d; ++c) o_row[c] /= Z * Z;"),
     "padded_length_used": ("long n = kv_lens ? (long)kv_lens[b] : (long)Tkv;", "long n = (long)Tkv;"),
-    "k_transposed_index": ("const uint16_t *kr = kb + j * (long)d;",
-                           "const uint16_t *kr = kb + (j % d) * (long)d;"),
+    "k_transposed_index": ("const long kr = kb + j * (long)d;",
+                           "const long kr = kb + (j % d) * (long)d;"),
+    # the E4M3 decoder of the FP8 K/V path
+    "e4m3_bias_8": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    "e4m3_subnormal_exponent": ("v = ldexp((double)m / 8.0, -6);", "v = ldexp((double)m / 8.0, -7);"),
+    "e4m3_no_nan_code": ("else if (e == 15 && m == 7)\n        return NAN;", "else if (0)\n        return NAN;"),
+    "fp8_v_scale_dropped": ("* s->v_scale", "* 1.0"),
+    "fp8_k_scale_on_v": ("e4m3_to_double(((const uint8_t *)s->v)[idx]) * s->v_scale",
+                         "e4m3_to_double(((const uint8_t *)s->v)[idx]) * s->k_scale"),
 }
 
 
@@ -416,6 +423,8 @@ def test_planted_mistakes_are_caught(mutation, tmp_path):
         lambda: _pin_padded(mod),
         lambda: _pin_constant_v(mod),
         lambda: _pin_brute(mod),
+        lambda: _pin_e4m3_table(mod),
+        lambda: _pin_fp8kv_equals_dequantised(mod),
     ]
     for pin in pins:
         try:
@@ -486,3 +495,97 @@ def _pin_brute(mod):
     bo, bl = _brute_force(q, k, v, kv, None, 0.45, True)
     np.testing.assert_allclose(o, bo, rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(l, bl, rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# FP8 (E4M3) K/V: the decoder and the attention on dequantised values
+# --------------------------------------------------------------------------
+
+# bytes whose values follow directly from the format definition (sign, 4-bit
+# exponent with bias 7, 3-bit mantissa; exponent field 0 is subnormal with
+# exponent -6; exponent 15 with mantissa 7 is NaN; no infinities)
+E4M3_HAND = {0x00: 0.0, 0x38: 1.0, 0xB8: -1.0, 0x3C: 1.5, 0x40: 2.0, 0x7E: 448.0, 0xFE: -448.0,
+             0x08: 2.0 ** -6, 0x07: 7 * 2.0 ** -9, 0x01: 2.0 ** -9, 0x30: 0.5, 0x77: 240.0}
+
+
+def _pin_e4m3_table(mod):
+    codes = np.array(sorted(E4M3_HAND), np.uint8)
+    np.testing.assert_array_equal(mod.e4m3_decode(codes), np.array([E4M3_HAND[c] for c in sorted(E4M3_HAND)]))
+    assert np.isnan(mod.e4m3_decode(np.array([0x7F, 0xFF], np.uint8))).all()
+
+
+def test_e4m3_decoder_hand_values():
+    _pin_e4m3_table(oracle)
+
+
+def test_e4m3_decoder_matches_torch_for_every_byte():
+    """The oracle's decoder, written from the format definition, against torch's
+    float8_e4m3fn -> float64 conversion (a library routine) on all 256 bytes."""
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_decode(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    same = (ours == ref) | (np.isnan(ours) & np.isnan(ref))
+    assert same.all(), codes[~same]
+
+
+def _fp8_case(seed, B=2, Hq=8, Hkv=2, Tq=3, Tkv=40, d=16):
+    g = torch.Generator().manual_seed(seed)
+    k8 = (torch.randn((B, Hkv, Tkv, d), generator=g) * 60).to(torch.float8_e4m3fn)
+    v8 = (torch.randn((B, Hkv, Tkv, d), generator=g) * 60).to(torch.float8_e4m3fn)
+    q = rnd((B, Hq, Tq, d), seed + 1)
+    return q, k8, v8
+
+
+def _pin_fp8kv_equals_dequantised(mod):
+    """With power-of-two scales every dequantised value is exactly a bf16, so the
+    FP8 K/V attention must equal the bf16 attention on those values."""
+    q, k8, v8 = _fp8_case(31)
+    ks, vs = 2.0 ** -6, 2.0 ** -5
+    kv = np.array([40, 17], np.int32)
+    sink = np.linspace(-1, 1, 8).astype(np.float32)
+    kd = torch.from_numpy(mod.e4m3_decode(k8) * ks).to(torch.bfloat16)
+    vd = torch.from_numpy(mod.e4m3_decode(v8) * vs).to(torch.bfloat16)
+    assert np.array_equal(kd.double().numpy(), mod.e4m3_decode(k8) * ks)  # exactly representable
+    o8, l8 = mod.attention_fp8kv(q, k8, v8, ks, vs, kv, sink, scale=0.3, causal=True)
+    ob, lb = mod.attention(q, kd, vd, kv, sink, scale=0.3, causal=True)
+    np.testing.assert_array_equal(o8, ob)
+    np.testing.assert_array_equal(l8, lb)
+
+
+def test_fp8kv_equals_bf16_on_dequantised_values():
+    _pin_fp8kv_equals_dequantised(oracle)
+
+
+def test_fp8kv_scales():
+    """v_scale multiplies O and leaves lse alone; k_scale acts as a factor of the
+    logit scale."""
+    q, k8, v8 = _fp8_case(33)
+    o1, l1 = oracle.attention_fp8kv(q, k8, v8, 0.01, 0.02, None, None, scale=0.5)
+    o2, l2 = oracle.attention_fp8kv(q, k8, v8, 0.01, 0.06, None, None, scale=0.5)
+    np.testing.assert_allclose(o2, 3 * o1, rtol=1e-13, atol=1e-15)
+    np.testing.assert_array_equal(l1, l2)
+    o3, l3 = oracle.attention_fp8kv(q, k8, v8, 0.03, 0.02, None, None, scale=0.5 / 3)
+    np.testing.assert_allclose(o3, o1, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(l3, l1, rtol=1e-12, atol=1e-12)
+
+
+def test_fp8kv_padded_nan_bytes_have_no_effect():
+    q, k8, v8 = _fp8_case(35)
+    kv = np.array([23, 40], np.int32)
+    o1, l1 = oracle.attention_fp8kv(q, k8, v8, 0.01, 0.02, kv, None, scale=0.5, causal=True)
+    k8n, v8n = k8.clone().view(torch.uint8), v8.clone().view(torch.uint8)
+    k8n[0, :, 23:] = 0x7F
+    v8n[0, :, 23:] = 0xFF
+    o2, l2 = oracle.attention_fp8kv(q, k8n, v8n, 0.01, 0.02, kv, None, scale=0.5, causal=True)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+
+
+def test_fp8kv_rows_entry_matches_full_entry():
+    q, k8, v8 = _fp8_case(37)
+    kv = np.array([40, 9], np.int32)
+    o, l = oracle.attention_fp8kv(q, k8, v8, 0.015, 0.025, kv, None, scale=0.4, causal=True)
+    rows = np.array([0, 5, 17, 30, 47], np.int64)
+    orow, lrow = oracle.attention_rows_fp8kv(q, k8, v8, 0.015, 0.025, kv, None, 0.4, True, rows)
+    np.testing.assert_array_equal(orow, o.reshape(-1, o.shape[-1])[rows])
+    np.testing.assert_array_equal(lrow, l.reshape(-1)[rows])

@@ -35,3 +35,26 @@ def test_pages_read_back_as_the_contiguous_cache(page_size):
     assert len(spare) >= 1
     for p in spare:
         assert torch.isnan(kc[p].float()).all() and torch.isnan(vc[p].float()).all()
+
+
+def test_fp8_input_recipe():
+    """FP8 K/V inputs: E4M3 bytes with one scale per tensor, amax / 448 over the
+    finite values; dequantised they stay within half an E4M3 step of the drawn
+    bf16 values, and the NaN padding stays NaN."""
+    import math
+
+    import torch
+
+    from gqa_attention_forward_flash_b200.synth import WORKLOADS, make_inputs, shrink
+    w = shrink(WORKLOADS["batched_decode_fp8kv"], B=3, Tkv=257)
+    inp = make_inputs(w)
+    assert inp.k8.dtype == torch.float8_e4m3fn and inp.v8.dtype == torch.float8_e4m3fn
+    for x, x8, sc in ((inp.k, inp.k8, inp.k_scale), (inp.v, inp.v8, inp.v_scale)):
+        xf = x.float()
+        fin = torch.isfinite(xf)
+        assert math.isclose(sc, float(xf[fin].abs().max()) / 448.0, rel_tol=1e-7)
+        deq = x8.float() * sc
+        assert torch.equal(torch.isnan(deq), ~fin)
+        # E4M3 keeps 3 mantissa bits: relative error at most 2^-4 for normal values
+        err = (deq[fin] - xf[fin]).abs()
+        assert bool((err <= xf[fin].abs() * 2.0 ** -4 + sc * 2.0 ** -10).all())
