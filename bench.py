@@ -65,7 +65,7 @@ def unit_work(w: Workload, n: int):
     """Algorithmic bytes and flops of one (batch, KV head) unit with length n."""
     pairs_per_head = sum(visible_keys(w, n, i) for i in range(w.Tq))
     keys = max((visible_keys(w, n, i) for i in range(w.Tq)), default=0)
-    kv_bytes = 2 * keys * w.d * 2
+    kv_bytes = 2 * keys * w.d * (1 if w.kv_fp8 else 2)  # E4M3 caches: one byte per element
     q_o_bytes = 2 * w.G * w.Tq * w.d * 2 + w.G * w.Tq * 4
     flops = 4 * w.d * pairs_per_head * w.G
     return kv_bytes + q_o_bytes, flops
@@ -223,8 +223,12 @@ def oracle_sample(w: Workload, inp, target_seconds: float, seed: int = 0):
             # a slice of the unit's rows: count exactly the work of those rows
             rows = sorted(rng.choice(rows, size=512, replace=False).tolist())
         t0 = time.perf_counter()
-        oracle.attention_rows(inp.q, inp.k, inp.v, inp.kv_lens, inp.sink, inp.scale, inp.causal,
-                              np.array(rows, np.int64))
+        if w.kv_fp8:
+            oracle.attention_rows_fp8kv(inp.q, inp.k8, inp.v8, inp.k_scale, inp.v_scale, inp.kv_lens, inp.sink,
+                                        inp.scale, inp.causal, np.array(rows, np.int64))
+        else:
+            oracle.attention_rows(inp.q, inp.k, inp.v, inp.kv_lens, inp.sink, inp.scale, inp.causal,
+                                  np.array(rows, np.int64))
         t_total += time.perf_counter() - t0
         n = lens[b]
         if len(rows) == max_rows_per_unit:
@@ -232,7 +236,7 @@ def oracle_sample(w: Workload, inp, target_seconds: float, seed: int = 0):
         else:
             pairs = sum(visible_keys(w, n, r % w.Tq) for r in rows)
             keys = max(visible_keys(w, n, r % w.Tq) for r in rows)
-            ub = 2 * keys * w.d * 2 + len(rows) * (2 * w.d * 2 + 4)
+            ub = 2 * keys * w.d * (1 if w.kv_fp8 else 2) + len(rows) * (2 * w.d * 2 + 4)
             uf = 4 * w.d * pairs
         done_b += ub
         done_f += uf
@@ -252,7 +256,8 @@ def run_reference(args, w, ws, rank):
         return
     inp = make_inputs(w)
     unit, _ = metric_unit(w)
-    per_step = max(0.5, args.ref_step_seconds)
+    # each step a bounded oracle sample; the whole run stays within about two minutes
+    per_step = max(0.3, min(args.ref_step_seconds, 120.0 / max(1, args.steps + args.warmup)))
     for s in range(args.warmup):
         oracle_sample(w, inp, per_step, seed=s)
     vals, times = [], []
@@ -277,6 +282,7 @@ def run_reference(args, w, ws, rank):
 
 def config_of(w: Workload, page_size: int = 0):
     c = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "G": w.G, "Tq": w.Tq, "Tkv": w.Tkv, "d": w.d,
+         "kv_dtype": "e4m3 (per-tensor scales)" if w.kv_fp8 else "bf16",
          "causal": w.causal, "sink": w.sink, "seed": w.seed,
          "kv_len": "U[1,%d]" % w.Tkv if w.ragged else (w.kv_len or w.Tkv),
          "nan_padding": w.nan_pad, "sigma": w.sigma,
@@ -299,7 +305,10 @@ def measure(args, w, ws, rank, local, steps, cpu_seconds, with_e2e=True):
     binding.load()
     dev = torch.device("cuda", local if ws > 1 else 0)
     inp = make_inputs(w)
-    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    if w.kv_fp8:
+        q, k, v = inp.q.to(dev), inp.k8.to(dev), inp.v8.to(dev)
+    else:
+        q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
     kv = None if inp.kv_lens is None else inp.kv_lens.to(dev)
     sink = None if inp.sink is None else inp.sink.to(dev)
     out = torch.empty_like(q)
@@ -316,6 +325,9 @@ def measure(args, w, ws, rank, local, steps, cpu_seconds, with_e2e=True):
         st = stream if st is None else st
         if args.page_size:
             binding.gqa_attention_fwd_paged(q, kc, vc, table, lens, sink, out, lse, scale=inp.scale,
+                                            causal=inp.causal, stream=st)
+        elif w.kv_fp8:
+            binding.gqa_attention_fwd_fp8kv(q, k, v, inp.k_scale, inp.v_scale, kv, sink, out, lse, scale=inp.scale,
                                             causal=inp.causal, stream=st)
         else:
             binding.gqa_attention_fwd(q, k, v, kv, sink, out, lse, scale=inp.scale, causal=inp.causal,
@@ -471,7 +483,8 @@ def run_e2e(args, w, inp, dev, stream, nbytes, nflops, ws):
         kc, vc, table, lens = paged_inputs(w, inp, args.page_size)
         hq, hk, hv, hkv, htab = (t.pin_memory() for t in (inp.q, kc, vc, lens, table))
     else:
-        hq, hk, hv = inp.q.pin_memory(), inp.k.pin_memory(), inp.v.pin_memory()
+        kk, vv = (inp.k8, inp.v8) if w.kv_fp8 else (inp.k, inp.v)
+        hq, hk, hv = inp.q.pin_memory(), kk.pin_memory(), vv.pin_memory()
         hkv = None if inp.kv_lens is None else inp.kv_lens.pin_memory()
         htab = None
     hs = None if inp.sink is None else inp.sink.pin_memory()
@@ -499,6 +512,9 @@ def run_e2e(args, w, inp, dev, stream, nbytes, nflops, ws):
         if paged:
             binding.gqa_attention_fwd_paged(dq, dk, dv, dtab, dkv, ds, dout, dlse, scale=inp.scale,
                                             causal=inp.causal, stream=stream)
+        elif w.kv_fp8:
+            binding.gqa_attention_fwd_fp8kv(dq, dk, dv, inp.k_scale, inp.v_scale, dkv, ds, dout, dlse,
+                                            scale=inp.scale, causal=inp.causal, stream=stream)
         else:
             binding.gqa_attention_fwd(dq, dk, dv, dkv, ds, dout, dlse, scale=inp.scale, causal=inp.causal,
                                       stream=stream)

@@ -28,6 +28,7 @@ SIGNATURES = {
     "gqa_attention_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "gqa_attention_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "gqa_attention_fwd_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "gqa_attention_fwd_fp8kv": (_I, [_P, _P, _P, _F, _F, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "gqa_attention_fwd_partial": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P, _P]),
     "gqa_splitkv_combine": (_I, [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
     "gqa_shard_lengths": (_I, [_P, _I, _I, _I, _P, _P]),
@@ -133,6 +134,38 @@ def gqa_attention_fwd_paged(q, k_cache, v_cache, page_table, kv_lens, sink=None,
                                         _ptr(sink), _ptr(out), _ptr(lse), B, Hq, Hkv, Tq, num_pages, page_size,
                                         max_pages, d, float(scale), int(bool(causal)), _stream(stream))
     _check("gqa_attention_fwd_paged", rc)
+    return out, lse
+
+
+def _need_e4m3(t, name, ndim):
+    if t.dtype not in (torch.float8_e4m3fn, torch.uint8) or t.dim() != ndim or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError("%s must be a contiguous CUDA float8_e4m3fn (or uint8) tensor with %d dims" % (name, ndim))
+
+
+def gqa_attention_fwd_fp8kv(q, k8, v8, k_scale, v_scale, kv_lens=None, sink=None, out=None, lse=None, scale=None,
+                            causal=False, stream=None):
+    """The forward on an FP8 K/V cache: K = k8 * k_scale, V = v8 * v_scale with
+    k8/v8 E4M3 [B,Hkv,Tkv,d] (float8_e4m3fn or their uint8 bytes) and per-tensor
+    scales.  q [B,Hq,Tq,d] bf16.  Returns (out, lse)."""
+    _need(q, torch.bfloat16, "q", 4)
+    _need_e4m3(k8, "k8", 4)
+    _need_e4m3(v8, "v8", 4)
+    B, Hq, Tq, d = q.shape
+    _, Hkv, Tkv, _ = k8.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=q.device)
+    if kv_lens is not None:
+        _need(kv_lens, torch.int32, "kv_lens", 1)
+    if sink is not None:
+        _need(sink, torch.float32, "sink", 1)
+    if scale is None:
+        scale = d ** -0.5
+    rc = load().gqa_attention_fwd_fp8kv(_ptr(q), _ptr(k8), _ptr(v8), float(k_scale), float(v_scale), _ptr(kv_lens),
+                                        _ptr(sink), _ptr(out), _ptr(lse), B, Hq, Hkv, Tq, Tkv, d, float(scale),
+                                        int(bool(causal)), _stream(stream))
+    _check("gqa_attention_fwd_fp8kv", rc)
     return out, lse
 
 

@@ -83,6 +83,19 @@ int get_state(DeviceState** out) {
     return GQA_OK;
 }
 
+// 2-D byte view [rows, cols] (E4M3 K/V) with a (cols x box_rows) box and the
+// 128-byte swizzle; cols = 128 bytes = one swizzle row.
+int make_tmap_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(cols), box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_CUDA;
+}
+
 // 2-D bf16 view [rows, cols] with a (64 x box_rows) box and the 128-byte swizzle.
 int make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
     cuuint64_t dims[2] = {cols, rows};
@@ -136,6 +149,8 @@ void fill_params(Params& p, int B, int Hq, int Hkv, int Tq, int Tkv, int d, floa
     p.out = reinterpret_cast<__nv_bfloat16*>(out);
     p.lse = lse;
     p.timeout_cycles = timeout;
+    p.kv_fp8 = 0;
+    p.v_scale = 1.f;
 }
 
 // Kernel configurations (shared-memory and TMEM budgets are checked in the Cfg
@@ -159,6 +174,9 @@ using CDec8 = DecCfg<8>;
 using CDec16 = DecCfg<16>;
 using CDec8_P = DecCfg<8, true>;
 using CDec16_P = DecCfg<16, true>;
+// the same over an E4M3 K/V cache (converted to f16 in shared memory)
+using CDec8_F8 = DecCfg<8, false, true>;
+using CDec16_F8 = DecCfg<16, false, true>;
 bool uses_decode_kernel(const Params& p) { return p.d == 128 && p.mode == 0 && p.R <= DEC_NQ; }
 // Head dims 256 and 512: the wide kernel (128-key tiles streamed in 64-column
 // chunks past a resident Q tile, in-kernel merge of split row-blocks).  At 512 a
@@ -223,15 +241,22 @@ int launch_fwd(const Params& p0, const void* q, const void* k, const void* v, in
         p.kv_box_rows = kvrows < static_cast<uint64_t>(C::BN) ? static_cast<int>(kvrows) : C::BN;
     int rc = make_tmap(&tq, q, qrows, C::D, p.q_box_rows);
     if (rc) return rc;
-    rc = make_tmap(&tk, k, kvrows, kvcols, p.kv_box_rows);
-    if (rc) return rc;
-    rc = make_tmap(&tv, v, kvrows, kvcols, p.kv_box_rows);
-    if (rc) return rc;
+    if constexpr (KIND == kDecode && C::FP8) {
+        rc = make_tmap_u8(&tk, k, kvrows, kvcols, p.kv_box_rows);
+        if (rc) return rc;
+        rc = make_tmap_u8(&tv, v, kvrows, kvcols, p.kv_box_rows);
+        if (rc) return rc;
+    } else {
+        rc = make_tmap(&tk, k, kvrows, kvcols, p.kv_box_rows);
+        if (rc) return rc;
+        rc = make_tmap(&tv, v, kvrows, kvcols, p.kv_box_rows);
+        if (rc) return rc;
+    }
     if (ev_before && cudaEventRecord(ev_before, stream) != cudaSuccess) return GQA_ERR_CUDA;
     if constexpr (KIND == kTwoLane)
         gqa_fwd2_kernel<C><<<grid, NUM_THREADS2, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     else if constexpr (KIND == kDecode)
-        gqa_dec_kernel<C><<<grid, NUM_THREADS_DEC, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+        gqa_dec_kernel<C><<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     else {
         // the stream-K merge waits for pieces written by other CTAs of the grid:
         // every CTA must be resident at once, which a cooperative launch guarantees
@@ -264,6 +289,9 @@ int dispatch_fwd(const Params& p, const void* q, const void* k, const void* v, i
                               : launch_fwd<C2_64_DQ, kTwoLane>(p, q, k, v, grid, stream, e0, e1);
         case 128:
             if (uses_decode_kernel(p)) {
+                if (p.kv_fp8)
+                    return p.R <= 8 ? launch_fwd<CDec8_F8, kDecode>(p, q, k, v, grid, stream, e0, e1)
+                                    : launch_fwd<CDec16_F8, kDecode>(p, q, k, v, grid, stream, e0, e1);
                 if (p.page_size > 0)
                     return p.R <= 8 ? launch_fwd<CDec8_P, kDecode>(p, q, k, v, grid, stream, e0, e1)
                                     : launch_fwd<CDec16_P, kDecode>(p, q, k, v, grid, stream, e0, e1);
@@ -402,6 +430,30 @@ extern "C" int gqa_attention_fwd(const void* q, const void* k, const void* v, co
     Params p;
     fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale, causal, kv_lens, sink, out, lse, 0, timeout_cycles(*s));
     return run_streamk(p, q, k, v, *s, stream);
+}
+
+extern "C" int gqa_attention_fwd_fp8kv(const void* q, const void* k8, const void* v8, float k_scale, float v_scale,
+                                       const int32_t* kv_lens, const float* sink, void* out, float* lse, int B, int Hq,
+                                       int Hkv, int Tq, int Tkv, int d, float scale, int causal, gqa_stream_t stream) {
+    int rc = check_common(q, k8, v8, B, Hq, Hkv, Tq, Tkv, d, scale);
+    if (rc) return rc;
+    if (!(k_scale > 0.f) || !std::isfinite(k_scale) || !(v_scale > 0.f) || !std::isfinite(v_scale)) return GQA_ERR_SHAPE;
+    // the swap-AB decode kernel's shapes: head dim 128, at most 16 packed rows per KV head
+    if (d != 128 || (Hq / Hkv) * static_cast<long long>(Tq) > DEC_NQ) return GQA_ERR_UNSUPPORTED;
+    if (!std::isfinite(scale * k_scale)) return GQA_ERR_SHAPE;
+    if (B == 0 || Tq == 0) return GQA_OK;
+    if (!out) return GQA_ERR_NULL;
+    if (!aligned16(out) || (lse && !aligned16(lse))) return GQA_ERR_ALIGN;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState* s = nullptr;
+    rc = get_state(&s);
+    if (rc) return rc;
+    if (s->cc_major != 10) return GQA_ERR_UNSUPPORTED;
+    Params p;
+    fill_params(p, B, Hq, Hkv, Tq, Tkv, d, scale * k_scale, causal, kv_lens, sink, out, lse, 0, timeout_cycles(*s));
+    p.kv_fp8 = 1;
+    p.v_scale = v_scale;
+    return run_streamk(p, q, k8, v8, *s, stream);
 }
 
 extern "C" int gqa_attention_fwd_paged(const void* q, const void* k_cache, const void* v_cache,

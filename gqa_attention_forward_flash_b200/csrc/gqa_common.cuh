@@ -62,6 +62,10 @@ struct Params {
     int page_size;
     int max_pages;
     int num_pages;
+    // FP8 K/V (swap-AB decode kernel): K/V are E4M3 bytes; k_scale is folded into
+    // scale_log2, v_scale multiplies the normalised output (1 otherwise)
+    int kv_fp8;
+    float v_scale;
 };
 
 // ------------------------------------------------------------------ schedule

@@ -24,7 +24,19 @@
 // MMA issuer, 3 split-segment ticket taker, 4-7 softmax (warp 4+q reads TMEM
 // lane quadrant q).  The stream-K work split, the split partial slots and the
 // last-arriver merge are those of the two-lane kernel (gqa_fwd2_kernel.cuh).
+//
+// FP8 K/V (FP8 = true; the AstrAI commit log's fp8 family stores tensors as E4M3
+// with one scale per tensor): each K/V tile arrives by TMA as 128 keys x 128
+// bytes in the upper half of its 32 KB stage, and four converter warps (8-11)
+// widen it in place to the f16 layout the MMAs read (E4M3 -> f16 is exact),
+// zeroing V rows past the logical length as they go; Q is converted from bf16
+// to f16 in place once per segment, and P' is written as f16, so both MMAs run
+// with f16 operands.  k_scale is folded into the logit scale and v_scale into
+// the output normalisation.
 #pragma once
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "gqa_fwd2_kernel.cuh"
 
 namespace gqa {
@@ -33,12 +45,15 @@ constexpr int NUM_THREADS_DEC = 256;
 constexpr int NSOFT_DEC = 128;
 constexpr int DEC_NQ = 16;  // N of both MMAs: packed query rows held (padded)
 
-template <int NR_, bool PAGED_ = false>
+template <int NR_, bool PAGED_ = false, bool FP8_ = false>
 struct DecCfg {
     static constexpr int D = 128, BN = 128, STK = 3, STV = 3, QBUF = 2;
     static constexpr int NR = NR_;  // query rows the softmax reads (8 or 16)
     static_assert(NR == 8 || NR == 16, "rows");
     static constexpr bool PAGED = PAGED_;
+    static constexpr bool FP8 = FP8_;  // K/V stored as E4M3 bytes (contiguous caches only)
+    static_assert(!(PAGED && FP8), "fp8 K/V over a paged cache is not built");
+    static constexpr int NTHREADS = FP8 ? 384 : 256;  // + four converter warps
     static constexpr int NBOX = D / 64;
     static constexpr int KV_BOX = BN * 128;             // one 64-column box of a K/V tile
     static constexpr int KV_BYTES = NBOX * KV_BOX;
@@ -66,7 +81,10 @@ struct DecCfg {
     static constexpr int B_FINAL = B_XSYNC + 1;
     static constexpr int B_MJOB = B_FINAL + 1;          // [2] partial rows of split segment j written
     static constexpr int B_MTICK = B_MJOB + 2;          // [2] ticket of split segment j taken
-    static constexpr int NBAR = B_MTICK + 2;
+    static constexpr int B_KCONV = B_MTICK + 2;         // [STK] FP8: K stage widened to f16
+    static constexpr int B_VCONV = B_KCONV + STK;       // [STV] FP8: V stage widened to f16
+    static constexpr int B_QCONV = B_VCONV + STV;       // [QBUF] FP8: Q buffer converted to f16
+    static constexpr int NBAR = B_QCONV + QBUF;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int MISC_BYTES = 1536;
     static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES;
@@ -74,9 +92,55 @@ struct DecCfg {
     static constexpr uint32_t TM_COLS = 64;
     static constexpr uint32_t TM_S = 0;   // + 16 * buffer
     static constexpr uint32_t TM_O = 32;
-    static constexpr uint32_t IDESC_S = ptx::umma_idesc_bf16_f32(BN, DEC_NQ, false, false);
-    static constexpr uint32_t IDESC_PV = ptx::umma_idesc_bf16_f32(D, DEC_NQ, true, false);
+    static constexpr uint32_t IDESC_S =
+        FP8 ? ptx::umma_idesc_f16_f32(BN, DEC_NQ, false, false) : ptx::umma_idesc_bf16_f32(BN, DEC_NQ, false, false);
+    static constexpr uint32_t IDESC_PV =
+        FP8 ? ptx::umma_idesc_f16_f32(D, DEC_NQ, true, false) : ptx::umma_idesc_bf16_f32(D, DEC_NQ, true, false);
+    // FP8: the raw E4M3 tile (128 keys x 128 bytes, 128-byte swizzle) lands in the
+    // upper half of its stage; widened, it fills the stage as two 64-column f16 boxes
+    static constexpr int KV_RAW_OFF = FP8 ? KV_BOX : 0;
+    static constexpr int RAW_TILE = BN * 128;
+    // the stages a role waits for before an MMA reads them
+    static constexpr int B_KREADY = FP8 ? B_KCONV : B_KFULL;
+    static constexpr int B_VREADY = FP8 ? B_VCONV : B_VFULL;
+    static constexpr int B_QREADY = FP8 ? B_QCONV : B_QFULL;
 };
+
+// Two E4M3 bytes (the first in the low byte) -> two f16 (the first in the low half).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xFFFFu), __NV_E4M3);
+    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+// FP8: widen one stage in place, 128 converter threads (ct = 0..127).  Raw byte
+// chunk c (16 keys' worth of columns 16c..16c+15) of row r sits at r*128 +
+// ((c ^ r%8) << 4) of the raw tile; its 16 f16 go to box c/4, chunks 2(c%4) and
+// 2(c%4)+1 of row r.  Box 1 overlaps the raw tile row for row, so each warp
+// reads its four rows completely before it writes them.  Rows >= zrow are
+// written as zeros.
+template <class C>
+__device__ __forceinline__ void dec_widen_stage(uint8_t* stage, int ct, int zrow) {
+    const uint8_t* raw = stage + C::KV_RAW_OFF;
+#pragma unroll 2
+    for (int k = 0; k < (C::BN * 8) / 128; ++k) {
+        const int i = ct + 128 * k;
+        const int r = i >> 3, c = i & 7;
+        const uint4 x = *reinterpret_cast<const uint4*>(raw + r * 128 + ((c ^ (r & 7)) << 4));
+        __syncwarp();
+        uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
+        if (r < zrow) {
+            lo = make_uint4(e4m3x2_to_f16x2(x.x), e4m3x2_to_f16x2(x.x >> 16), e4m3x2_to_f16x2(x.y),
+                            e4m3x2_to_f16x2(x.y >> 16));
+            hi = make_uint4(e4m3x2_to_f16x2(x.z), e4m3x2_to_f16x2(x.z >> 16), e4m3x2_to_f16x2(x.w),
+                            e4m3x2_to_f16x2(x.w >> 16));
+        }
+        uint8_t* row = stage + (c >> 2) * C::KV_BOX + r * 128;
+        const int c2 = 2 * (c & 3);
+        *reinterpret_cast<uint4*>(row + ((c2 ^ (r & 7)) << 4)) = lo;
+        *reinterpret_cast<uint4*>(row + (((c2 + 1) ^ (r & 7)) << 4)) = hi;
+        __syncwarp();
+    }
+}
 
 struct DecMisc {
     uint32_t tmem_base;       // the first four fields match Misc (bounded waits read abort)
@@ -139,7 +203,7 @@ __device__ __noinline__ bool dec_issue_pv(const Params& p, Misc* wmisc, uint32_t
     auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
     const int st = gg % C::STV;
     if (!wait_bar(bar(C::B_PFULL + (gg & 1u)), (gg >> 1) & 1u, wmisc, p)) return false;
-    if (!wait_bar(bar(C::B_VFULL + st), (gg / C::STV) & 1u, wmisc, p)) return false;
+    if (!wait_bar(bar(C::B_VREADY + st), (gg / C::STV) & 1u, wmisc, p)) return false;
     if (first && seg > 0 && !wait_bar(bar(C::B_OFREE), (seg - 1) & 1, wmisc, p)) return false;
     ptx::tc_fence_after();
     const uint32_t vbase = sbase + C::OFF_V + st * C::KV_BYTES;
@@ -156,7 +220,7 @@ __device__ __noinline__ bool dec_issue_pv(const Params& p, Misc* wmisc, uint32_t
 }
 
 template <class C>
-__global__ void __launch_bounds__(NUM_THREADS_DEC, 1)
+__global__ void __launch_bounds__(C::NTHREADS, 1)
 gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const Params p) {
     constexpr int NR = C::NR;
@@ -198,6 +262,9 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ptx::mbar_init(bar(C::B_MJOB + i), 1);
             ptx::mbar_init(bar(C::B_MTICK + i), 1);
         }
+        for (int i = 0; i < C::STK; ++i) ptx::mbar_init(bar(C::B_KCONV + i), 4);
+        for (int i = 0; i < C::STV; ++i) ptx::mbar_init(bar(C::B_VCONV + i), 4);
+        for (int i = 0; i < C::QBUF; ++i) ptx::mbar_init(bar(C::B_QCONV + i), 4);
         ptx::mbar_init(bar(C::B_OFREE), 4);
         ptx::mbar_init(bar(C::B_RED), 4);
         ptx::mbar_init(bar(C::B_XSYNC), 4);
@@ -214,7 +281,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ptx::tmem_relinquish();
     }
     if (warp == 0) plan_span(p, cta, NC, &misc->span);
-    if (warp >= 4) {
+    if (warp >= 4 && warp < 8) {
         // P' rows past NR are never written by the softmax: keep them zero
         uint4* pz = reinterpret_cast<uint4*>(smem + C::OFF_P);
         for (int i = threadIdx.x - 128; i < 2 * C::P_BYTES / 16; i += NSOFT_DEC) pz[i] = make_uint4(0, 0, 0, 0);
@@ -256,8 +323,15 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     ok = wait_bar(bar(C::B_KEMPTY + st), ((g / C::STK) & 1) ^ 1, wmisc, p);
                     if (!ok) break;
                     ++k_issued[st];
-                    load_kv_tile<C>(p, &tm_k, sbase + C::OFF_K + st * C::KV_BYTES, bar(C::B_KFULL + st), rb, t, sg.n,
-                                    pol_kv);
+                    if constexpr (C::FP8) {
+                        ptx::mbar_arrive_expect_tx(bar(C::B_KFULL + st), p.kv_box_rows * 128);
+                        ptx::tma_load_2d(sbase + C::OFF_K + st * C::KV_BYTES + C::KV_RAW_OFF, &tm_k, 0,
+                                         static_cast<int>(rb.kv_row0 + static_cast<long long>(t) * C::BN),
+                                         bar(C::B_KFULL + st), pol_kv);
+                    } else {
+                        load_kv_tile<C>(p, &tm_k, sbase + C::OFF_K + st * C::KV_BYTES, bar(C::B_KFULL + st), rb, t,
+                                        sg.n, pol_kv);
+                    }
                 }
                 ++seg_i;
             }
@@ -282,8 +356,15 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     ok = wait_bar(bar(C::B_VEMPTY + st), ((g / C::STV) & 1) ^ 1, wmisc, p);
                     if (!ok) break;
                     ++v_issued[st];
-                    load_kv_tile<C>(p, &tm_v, sbase + C::OFF_V + st * C::KV_BYTES, bar(C::B_VFULL + st), rb, t, sg.n,
-                                    pol_kv);
+                    if constexpr (C::FP8) {
+                        ptx::mbar_arrive_expect_tx(bar(C::B_VFULL + st), p.kv_box_rows * 128);
+                        ptx::tma_load_2d(sbase + C::OFF_V + st * C::KV_BYTES + C::KV_RAW_OFF, &tm_v, 0,
+                                         static_cast<int>(rb.kv_row0 + static_cast<long long>(t) * C::BN),
+                                         bar(C::B_VFULL + st), pol_kv);
+                    } else {
+                        load_kv_tile<C>(p, &tm_v, sbase + C::OFF_V + st * C::KV_BYTES, bar(C::B_VFULL + st), rb, t,
+                                        sg.n, pol_kv);
+                    }
                 }
             }
             for (int i = 0; i < C::STV; ++i) drain_bar(bar(C::B_VFULL + i), v_issued[i], p.timeout_cycles);
@@ -324,12 +405,12 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     have_prev = false;
                 }
                 const int qb = seg_i % C::QBUF;
-                ok = wait_bar(bar(C::B_QFULL + qb), (seg_i / C::QBUF) & 1, wmisc, p);
+                ok = wait_bar(bar(C::B_QREADY + qb), (seg_i / C::QBUF) & 1, wmisc, p);
                 if (!ok) break;
                 const uint32_t qbase = sbase + C::OFF_Q + qb * C::Q_BYTES;
                 for (int t = sg.t0; t < sg.t1 && ok; ++t, ++g) {
                     const int stk = g % C::STK;
-                    ok = wait_bar(bar(C::B_KFULL + stk), (g / C::STK) & 1, wmisc, p);
+                    ok = wait_bar(bar(C::B_KREADY + stk), (g / C::STK) & 1, wmisc, p);
                     if (!ok) break;
                     ptx::tc_fence_after();
                     issue_s(g, qbase, sbase + C::OFF_K + stk * C::KV_BYTES);
@@ -373,7 +454,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
     }
     // ---------------------------------------------------------------- softmax warps
-    else {
+    else if (warp < 8) {
         const int quad = warp & 3;
         const int kl = quad * 32 + lane;  // key of the tile = S' lane; head dim = O' lane
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
@@ -502,10 +583,14 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     const float mu = (m_run[r] == -INFINITY) ? 0.f : m_run[r];
                     const float pr = ptx::ex2(x[r] - mu);
                     l_t[r] += pr;
-                    *reinterpret_cast<__nv_bfloat16*>(pb + r * 128 + ((pkey_chunk ^ (r & 7)) << 4)) = __float2bfloat16_rn(pr);
+                    if constexpr (C::FP8)
+                        *reinterpret_cast<__half*>(pb + r * 128 + ((pkey_chunk ^ (r & 7)) << 4)) = __float2half_rn(pr);
+                    else
+                        *reinterpret_cast<__nv_bfloat16*>(pb + r * 128 + ((pkey_chunk ^ (r & 7)) << 4)) = __float2bfloat16_rn(pr);
                 }
-                // padded key rows of the V tile reach the MMA as zeros (0 * NaN = NaN)
-                if ((t + 1) * C::BN > sg.n) {
+                // padded key rows of the V tile reach the MMA as zeros (0 * NaN = NaN);
+                // with FP8 K/V the converter warps write them as zeros
+                if (!C::FP8 && (t + 1) * C::BN > sg.n) {
                     const int st = g % C::STV;
                     bool okv = wait_bar(bar(C::B_VFULL + st), (g / C::STV) & 1, wmisc, p);
                     okv = __all_sync(0xffffffffu, okv);
@@ -572,7 +657,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         const float a = (el[r] > 0.f) ? ptx::ex2(em[r] - M) : 0.f;
                         const float lt = el[r] * a + ((sk != -INFINITY) ? ptx::ex2(sk - M) : 0.f);
                         if (lt > 0.f) {
-                            w = a / lt;
+                            w = a / lt * p.v_scale;
                             lse_v = (M + __log2f(lt)) * LN2;
                         }
                     }
@@ -580,7 +665,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     if (kl == 0 && p.lse != nullptr) p.lse[fr] = lse_v;
                 } else {
                     if (el[r] > 0.f) {
-                        w = 1.f / el[r];
+                        w = p.v_scale / el[r];
                         lse_v = (em[r] + __log2f(el[r])) * LN2;
                     }
                     const long long prow = static_cast<long long>(sg.slot) * BM + r;
@@ -698,6 +783,56 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (r < rb.rows_valid) p.out[(rb.q_row0 + r) * C::D + kl] = __float2bfloat16_rn(acc[r]);
             if (stid == 0) p.counters[sgm.w] = 0;
             if (!xsync()) { ok = false; break; }
+        }
+    }
+
+    // ---------------------------------------------------------------- FP8 converter warps
+    else if constexpr (C::FP8) {
+        const int ct = threadIdx.x - 256;  // 0..127
+        SegWalker wk;
+        wk.init(p, misc->span, cta);
+        Seg sg;
+        int seg_i = 0;
+        uint32_t g = 0;
+        bool ok = true;
+        while (ok && wk.next(p, sg)) {
+            if (sg.t1 <= sg.t0) continue;
+            // Q: bf16 -> f16 in place (same layout)
+            const int qb = seg_i % C::QBUF;
+            ok = __all_sync(0xffffffffu, wait_bar(bar(C::B_QFULL + qb), (seg_i / C::QBUF) & 1, wmisc, p));
+            if (!ok) break;
+            uint4* qv = reinterpret_cast<uint4*>(smem + C::OFF_Q + qb * C::Q_BYTES);
+            for (int i = ct; i < C::Q_BYTES / 16; i += 128) {
+                uint4 x = qv[i];
+                uint32_t* w4 = reinterpret_cast<uint32_t*>(&x);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[j]));
+                    const __half2 h = __floats2half2_rn(f.x, f.y);
+                    w4[j] = *reinterpret_cast<const uint32_t*>(&h);
+                }
+                qv[i] = x;
+            }
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(C::B_QCONV + qb));
+            for (int t = sg.t0; t < sg.t1 && ok; ++t, ++g) {
+                const int stk = g % C::STK, stv = g % C::STV;
+                ok = __all_sync(0xffffffffu, wait_bar(bar(C::B_KFULL + stk), (g / C::STK) & 1, wmisc, p));
+                if (!ok) break;
+                dec_widen_stage<C>(smem + C::OFF_K + stk * C::KV_BYTES, ct, C::BN);
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar(C::B_KCONV + stk));
+                ok = __all_sync(0xffffffffu, wait_bar(bar(C::B_VFULL + stv), (g / C::STV) & 1, wmisc, p));
+                if (!ok) break;
+                // rows at or past the logical length reach the MMA as zeros (0 * NaN = NaN)
+                dec_widen_stage<C>(smem + C::OFF_V + stv * C::KV_BYTES, ct, sg.n - t * C::BN);
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar(C::B_VCONV + stv));
+            }
+            ++seg_i;
         }
     }
 

@@ -42,6 +42,7 @@ template <int D_, int STK_, int STV_, int RBQ_, bool PAGED_ = false>
 struct Fwd2Cfg {
     static constexpr int D = D_, BN = 128, STK = STK_, STV = STV_, RBQ = RBQ_;
     static constexpr bool PAGED = PAGED_;  // K/V from a paged cache (chosen at compile time)
+    static constexpr bool FP8 = false;     // bf16 K/V
     static_assert(D == 64 || D == 128, "head dim");
     static constexpr int NBOX = D / 64;
     static constexpr int Q_BOX = BM * 128;

@@ -64,6 +64,7 @@ template <int D_, int DSPLIT_>
 struct WideCfg {
     static constexpr int D = D_, DSPLIT = DSPLIT_, BN = 128;
     static constexpr int DO = D / DSPLIT;  // O columns held by one CTA
+    static constexpr bool FP8 = false;     // bf16 K/V
     static_assert((D == 256 && DSPLIT == 1) || (D == 512 && DSPLIT == 2), "head dim");
     static_assert(DO == 256, "O takes 256 TMEM columns");
     static constexpr int NBOX = D / 64;   // K chunks per tile (and Q boxes)

@@ -17,7 +17,8 @@
 //      SBO = 1024 (stride between groups of 8 K-rows), LBO = stride between
 //      64-wide MN blocks.
 //  * UMMA instruction descriptor (kind::f16): D format F32 (bit 4), A and B
-//    format BF16 (bits 7, 10), A/B major in bits 15/16 (1 = MN-major), N >> 3 in
+//    format in bits 7-9 / 10-12 (0 = F16, 1 = BF16; both operands of one MMA
+//    have the same type), A/B major in bits 15/16 (1 = MN-major), N >> 3 in
 //    bits 17-22, M >> 4 in bits 24-28.
 //  * TMEM address: lane in bits 16-31, column in bits 0-15.  With M = 128 and
 //    one CTA, accumulator row i lives in lane i; warp w of a warpgroup may only
@@ -199,6 +200,14 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N, bool a_
     return (1u << 4)                                   // D: f32
            | (1u << 7)                                 // A: bf16
            | (1u << 10)                                // B: bf16
+           | (static_cast<uint32_t>(a_mn_major) << 15)  //
+           | (static_cast<uint32_t>(b_mn_major) << 16)  //
+           | (static_cast<uint32_t>(N >> 3) << 17)     //
+           | (static_cast<uint32_t>(M >> 4) << 24);
+}
+// The same with A and B both f16 (format field 0).
+__host__ __device__ constexpr uint32_t umma_idesc_f16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+    return (1u << 4)                                   // D: f32
            | (static_cast<uint32_t>(a_mn_major) << 15)  //
            | (static_cast<uint32_t>(b_mn_major) << 16)  //
            | (static_cast<uint32_t>(N >> 3) << 17)     //

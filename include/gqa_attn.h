@@ -187,6 +187,28 @@ int gqa_attention_fwd_paged(const void *q, const void *k_cache, const void *v_ca
                             int causal, gqa_stream_t stream);
 
 /*
+ * gqa_attention_fwd with the K/V cache stored in FP8: OCP E4M3 bytes (sign,
+ * 4-bit exponent with bias 7, 3-bit mantissa, no infinities) with one scale per
+ * tensor, the storage of the AstrAI commit log's fp8 family (e4m3 quantize with
+ * a per-tensor scale from the tensor's amax; the consumer multiplies back by
+ * the scale).  The attention above is computed on
+ *   K = value(k8) * k_scale,   V = value(v8) * v_scale.
+ *   k8, v8:  uint8 [B, Hkv, Tkv, d] E4M3 bytes, contiguous, 16-byte aligned;
+ *            rows past kv_lens[b] may hold anything (NaN included)
+ *   k_scale, v_scale: positive finite (else GQA_ERR_SHAPE)
+ * q, kv_lens, sink, out, lse, scale, causal as in gqa_attention_fwd.  Served
+ * for the decode shapes of the swap-AB kernel: d = 128 with G*Tq <= 16 packed
+ * query rows per KV head (GQA_ERR_UNSUPPORTED otherwise).  K/V tiles are read
+ * as bytes (half the HBM traffic of bf16) and widened exactly to f16 in shared
+ * memory; Q is taken to f16 (exact for |q| in [2^-14, 65504]) and P is kept in
+ * f16, so the tolerance of the bf16 path against the oracle on the dequantised
+ * K/V holds.  Scratch, errors and graph capture as in gqa_attention_fwd.
+ */
+int gqa_attention_fwd_fp8kv(const void *q, const void *k8, const void *v8, float k_scale, float v_scale,
+                            const int32_t *kv_lens, const float *sink, void *out, float *lse, int B, int Hq,
+                            int Hkv, int Tq, int Tkv, int d, float scale, int causal, gqa_stream_t stream);
+
+/*
  * gqa_attention_fwd without any device allocation.  The pages have no
  * counterpart to this entry point; it exists for callers that cannot let a
  * library allocate device memory: engines that carve all of HBM into their own

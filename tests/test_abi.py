@@ -159,3 +159,15 @@ def test_binding_wrappers_validate_before_calling(lib):
         binding.gqa_attention_fwd_noalloc(q, k, k)
     with pytest.raises(ValueError):
         binding.gqa_attention_fwd(q, k, k, kv_lens=torch.zeros(1, dtype=i32))
+
+
+def test_fp8kv_entry_rejects_bad_arguments_on_the_host(lib):
+    f = lib.gqa_attention_fwd_fp8kv
+    args = lambda ks=1.0, vs=1.0, d=128, Hq=8, Tq=1: (P(16), P(16), P(16), ks, vs, None, None, P(16), P(16), 1, Hq, 1,
+                                                      Tq, 8, d, 0.125, 0, None)
+    assert f(*args(ks=0.0)) == -2
+    assert f(*args(vs=-1.0)) == -2
+    assert f(*args(ks=float("inf"))) == -2
+    assert f(*args(d=64)) == -7
+    assert f(*args(Hq=32)) == -7      # 32 packed rows: not a decode shape
+    assert f(*args(Tq=3)) == -7       # 8 heads x 3 rows = 24 packed rows
