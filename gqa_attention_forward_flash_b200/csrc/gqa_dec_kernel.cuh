@@ -146,7 +146,7 @@ struct DecMisc {
     uint32_t tmem_base;       // the first four fields match Misc (bounded waits read abort)
     volatile int abort;
     volatile int merge_flag;
-    int npro;                 // first-segment tiles whose K and V the prologue issued
+    int pad;
     SpanStart span;
     float red[2][DEC_NQ][4];  // per-tile row reductions: [phase][row][softmax warp]
     float mlse[DEC_NQ];       // merged lse per packed row (in-kernel merge)
@@ -280,48 +280,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ptx::tmem_alloc(ptx::smem_addr(&misc->tmem_base), C::TM_COLS);
         ptx::tmem_relinquish();
     }
-    if (warp == 0) {
-        plan_span(p, cta, NC, &misc->span);
-        __syncwarp();
-        // Prologue: the thread that set up the barriers issues the first segment's Q
-        // and its first K and V tiles right after the plan, before the CTA barrier,
-        // so that the first loads leave while the roles' code is still being fetched.
-        if (lane == 0) {
-            int npro = 0;
-            SegWalker wk;
-            wk.init(p, misc->span, cta);
-            Seg sg;
-            if (!C::PAGED && wk.next(p, sg) && sg.t1 > sg.t0) {
-                const RB rb = rb_of(p, sg.w);
-                const uint64_t pol_q = ptx::policy_evict_last();
-                const uint64_t pol_kv = ptx::policy_evict_first();
-                ptx::mbar_arrive_expect_tx(bar(C::B_QFULL), C::NBOX * p.q_box_rows * 128);
-                for (int bx = 0; bx < C::NBOX; ++bx)
-                    ptx::tma_load_2d(sbase + C::OFF_Q + bx * C::Q_BOX, &tm_q, bx * 64, static_cast<int>(rb.q_row0),
-                                     bar(C::B_QFULL), pol_q);
-                npro = sg.t1 - sg.t0;
-                npro = npro < C::STK ? npro : C::STK;
-                npro = npro < C::STV ? npro : C::STV;
-                for (int i = 0; i < npro; ++i) {
-                    const int y = static_cast<int>(rb.kv_row0 + static_cast<long long>(sg.t0 + i) * C::BN);
-                    if constexpr (C::FP8) {
-                        ptx::mbar_arrive_expect_tx(bar(C::B_KFULL + i), p.kv_box_rows * 128);
-                        ptx::tma_load_2d(sbase + C::OFF_K + i * C::KV_BYTES + C::KV_RAW_OFF, &tm_k, 0, y,
-                                         bar(C::B_KFULL + i), pol_kv);
-                        ptx::mbar_arrive_expect_tx(bar(C::B_VFULL + i), p.kv_box_rows * 128);
-                        ptx::tma_load_2d(sbase + C::OFF_V + i * C::KV_BYTES + C::KV_RAW_OFF, &tm_v, 0, y,
-                                         bar(C::B_VFULL + i), pol_kv);
-                    } else {
-                        load_kv_tile<C>(p, &tm_k, sbase + C::OFF_K + i * C::KV_BYTES, bar(C::B_KFULL + i), rb,
-                                        sg.t0 + i, sg.n, pol_kv);
-                        load_kv_tile<C>(p, &tm_v, sbase + C::OFF_V + i * C::KV_BYTES, bar(C::B_VFULL + i), rb,
-                                        sg.t0 + i, sg.n, pol_kv);
-                    }
-                }
-            }
-            misc->npro = npro;
-        }
-    }
+    if (warp == 0) plan_span(p, cta, NC, &misc->span);
     if (warp >= 4 && warp < 8) {
         // P' rows past NR are never written by the softmax: keep them zero
         uint4* pz = reinterpret_cast<uint4*>(smem + C::OFF_P);
@@ -348,28 +307,19 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             uint32_t k_issued[C::STK], q_issued[C::QBUF];
             for (int i = 0; i < C::STK; ++i) k_issued[i] = 0;
             for (int i = 0; i < C::QBUF; ++i) q_issued[i] = 0;
-            const int npro = misc->npro;  // the prologue issued Q and these first tiles
             while (ok && wk.next(p, sg)) {
                 if (sg.t1 <= sg.t0) continue;
                 const RB rb = rb_of(p, sg.w);
                 const int qb = seg_i % C::QBUF;
-                if (seg_i == 0 && npro > 0) {
-                    ++q_issued[qb];
-                } else {
-                    ok = wait_bar(bar(C::B_QEMPTY + qb), ((seg_i / C::QBUF) & 1) ^ 1, wmisc, p);
-                    if (!ok) break;
-                    ptx::mbar_arrive_expect_tx(bar(C::B_QFULL + qb), C::NBOX * p.q_box_rows * 128);
-                    ++q_issued[qb];
-                    for (int bx = 0; bx < C::NBOX; ++bx)
-                        ptx::tma_load_2d(sbase + C::OFF_Q + qb * C::Q_BYTES + bx * C::Q_BOX, &tm_q, bx * 64,
-                                         static_cast<int>(rb.q_row0), bar(C::B_QFULL + qb), pol_q);
-                }
+                ok = wait_bar(bar(C::B_QEMPTY + qb), ((seg_i / C::QBUF) & 1) ^ 1, wmisc, p);
+                if (!ok) break;
+                ptx::mbar_arrive_expect_tx(bar(C::B_QFULL + qb), C::NBOX * p.q_box_rows * 128);
+                ++q_issued[qb];
+                for (int bx = 0; bx < C::NBOX; ++bx)
+                    ptx::tma_load_2d(sbase + C::OFF_Q + qb * C::Q_BYTES + bx * C::Q_BOX, &tm_q, bx * 64,
+                                     static_cast<int>(rb.q_row0), bar(C::B_QFULL + qb), pol_q);
                 for (int t = sg.t0; t < sg.t1; ++t, ++g) {
                     const int st = g % C::STK;
-                    if (static_cast<int>(g) < npro) {
-                        ++k_issued[st];
-                        continue;
-                    }
                     ok = wait_bar(bar(C::B_KEMPTY + st), ((g / C::STK) & 1) ^ 1, wmisc, p);
                     if (!ok) break;
                     ++k_issued[st];
@@ -398,16 +348,11 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             bool ok = true;
             uint32_t v_issued[C::STV];
             for (int i = 0; i < C::STV; ++i) v_issued[i] = 0;
-            const int npro = misc->npro;
             while (ok && wk.next(p, sg)) {
                 if (sg.t1 <= sg.t0) continue;
                 const RB rb = rb_of(p, sg.w);
                 for (int t = sg.t0; t < sg.t1; ++t, ++g) {
                     const int st = g % C::STV;
-                    if (static_cast<int>(g) < npro) {
-                        ++v_issued[st];
-                        continue;
-                    }
                     ok = wait_bar(bar(C::B_VEMPTY + st), ((g / C::STV) & 1) ^ 1, wmisc, p);
                     if (!ok) break;
                     ++v_issued[st];
