@@ -188,11 +188,25 @@ using CW512 = WideCfg<512, 2>;
 int dsplit_for(int d) { return d == 512 ? CW512::DSPLIT : 1; }
 
 // Tile geometry of the kernel that will serve these sizes.
+// Extra weight (in key tiles) of a row-block start when the swap-AB decode
+// kernel cuts the work into spans: a segment's epilogue, switch and merge share
+// against a tile's streaming time.  Measured on the batched decode (B = 16, ragged
+// lengths): 7 tiles for bf16 K/V (1.25 us per tile; 85 -> 78 us against equal
+// spans), 2 for E4M3 K/V (its tiles take 1.75 us; 79 -> 69 us).
+int seg_weight(bool fp8) {
+    if (const char* e = std::getenv("GQA_SEG_WEIGHT")) {
+        const int v = std::atoi(e);
+        if (v >= 0 && v <= 64) return v;
+    }
+    return fp8 ? 2 : 7;
+}
+
 void choose_geometry(Params& p) {
     p.BN = 128;
     p.RBQ = (p.d <= 128 && p.R > BM) ? 2 : 1;
     p.QW = (p.QT + p.RBQ - 1) / p.RBQ;
     p.W = static_cast<long long>(p.U) * p.QW;
+    p.seg_w = (p.d == 128 && p.R <= DEC_NQ && p.B <= kMaxWeightedB) ? seg_weight(p.kv_fp8 != 0) : 0;
 }
 
 // Kernel families: the wide kernel (head dims 256, 512), the two-lane kernel

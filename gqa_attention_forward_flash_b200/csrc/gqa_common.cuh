@@ -22,6 +22,7 @@
 namespace gqa {
 
 constexpr int BM = 128;          // packed query rows per tile = TMEM lanes
+constexpr int kMaxGrid = 512;    // CTAs (or CTA groups) of a stream-K launch at most
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
@@ -66,6 +67,11 @@ struct Params {
     // scale_log2, v_scale multiplies the normalised output (1 otherwise)
     int kv_fp8;
     float v_scale;
+    // cost-weighted spans (swap-AB decode kernel): every row-block start counts as
+    // seg_w extra tiles when the flat order is cut into equal spans, so that a CTA
+    // whose span crosses more row-blocks (more epilogues, merges, segment
+    // switches) gets fewer tiles; 0 = equal spans of tiles
+    int seg_w;
 };
 
 // ------------------------------------------------------------------ schedule
@@ -265,6 +271,97 @@ __device__ void plan_span(const Params& p, int c, int NC, SpanStart* out) {
         out->w = w;
         out->t = t;
     }
+}
+
+// Cost-weighted spans (row-blocks of one q-tile: QW == 1).  Unit u = (b, g) has
+// nt(b) tiles and counts as E + nt(b) in weighted positions (E = p.seg_w): its
+// weighted extent [Y(u), Y(u) + E + nt(b)) with Y(u) = T(u) + u*E, T(u) its first
+// flat tile.  CTA c owns the weighted interval [c*tot_w/NC, (c+1)*tot_w/NC); a
+// weighted position y inside unit u maps to the flat tile T(u) + max(0, y - Y(u) - E)
+// (the first E positions of a unit carry its start-up cost and no tile).
+//
+// yb[b] (b = 0..B) is the weighted start of batch b's first unit, built by one
+// warp; from it, one thread maps boundary k to the flat start of CTA k's span
+// (and, for the CTA's own start, its row-block and tile).
+constexpr int kMaxWeightedB = 1024;  // batches the weighted plan keeps in its table
+
+__device__ int weighted_bound(const Params& p, const int* yb, int NC, int k, int* w_out, int* t_out) {
+    const long long E = p.seg_w;
+    const long long tot_w = yb[p.B];
+    const long long tot = tot_w - static_cast<long long>(p.B) * p.Hkv * E;
+    const long long y = (static_cast<long long>(k) * tot_w) / NC;
+    if (y >= tot_w) {
+        *w_out = 0;
+        *t_out = 0;
+        return static_cast<int>(tot);
+    }
+    int lo = 0, hi = p.B;  // yb[lo] <= y < yb[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (yb[mid] <= y) lo = mid;
+        else hi = mid;
+    }
+    const int per_unit = (yb[lo + 1] - yb[lo]) / p.Hkv;  // E + nt(b)
+    const int n = per_unit - static_cast<int>(E);
+    const int off = static_cast<int>(y - yb[lo]);
+    const int g = off / per_unit, r = off - g * per_unit;
+    const int t = r > E ? r - static_cast<int>(E) : 0;
+    *w_out = lo * p.Hkv + g;
+    *t_out = t;
+    return static_cast<int>(yb[lo] - static_cast<long long>(lo) * p.Hkv * E) + g * n + t;
+}
+
+// One full warp: the batch table yb[0..B] and this CTA's SpanStart.
+__device__ void plan_span_weighted(const Params& p, int c, int NC, SpanStart* out, int* yb) {
+    const int lane = threadIdx.x & 31;
+    const int E = p.seg_w;
+    int acc = 0;
+    for (int base = 0; base < p.B; base += 32) {
+        const int bb = base + lane;
+        const int lw = bb < p.B ? p.Hkv * (qtile_ntiles(p, 0, load_len(p, bb)) + E) : 0;
+        int inc = lw;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        if (bb < p.B) yb[bb] = acc + inc - lw;
+        acc += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (lane == 0) yb[p.B] = acc;
+    __syncwarp();
+    // lanes 0 and 1: the two boundaries of this CTA's span
+    int w = 0, t = 0, f = 0;
+    if (lane < 2) f = weighted_bound(p, yb, NC, c + lane, &w, &t);
+    const int f1 = __shfl_sync(0xffffffffu, f, 1);
+    if (lane == 0) {
+        out->tot = acc - static_cast<long long>(p.B) * p.Hkv * E;
+        out->p0 = f;
+        out->p1 = f1;
+        out->w = w;
+        out->t = t;
+    }
+}
+
+// One full warp: bounds[k] = flat start of CTA k's span, k = 0..NC.
+__device__ void fill_span_bounds(const Params& p, const int* yb, int NC, int* bounds) {
+    const int lane = threadIdx.x & 31;
+    for (int k = lane; k <= NC; k += 32) {
+        int w, t;
+        bounds[k] = weighted_bound(p, yb, NC, k, &w, &t);
+    }
+    __syncwarp();
+}
+
+// Owner of flat tile x under a bounds table: the last c with bounds[c] <= x.
+__device__ __forceinline__ int cta_of_table(const int* bounds, int NC, long long x) {
+    int lo = 0, hi = NC;  // bounds[lo] <= x < bounds[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (bounds[mid] <= x) lo = mid;
+        else hi = mid;
+    }
+    return lo;
 }
 
 // Walks this CTA's segments; every role keeps its own walker and all see the

@@ -84,9 +84,12 @@ struct DecCfg {
     static constexpr int B_KCONV = B_MTICK + 2;         // [STK] FP8: K stage widened to f16
     static constexpr int B_VCONV = B_KCONV + STK;       // [STV] FP8: V stage widened to f16
     static constexpr int B_QCONV = B_VCONV + STV;       // [QBUF] FP8: Q buffer converted to f16
-    static constexpr int NBAR = B_QCONV + QBUF;
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr int MISC_BYTES = 1536;
+    static constexpr int B_BOUNDS = B_QCONV + QBUF;     // the span bounds table is filled
+    static constexpr int NBAR = B_BOUNDS + 1;
+    // the control block holds float4-read arrays: 128-byte aligned whatever NBAR is
+    static constexpr int OFF_MISC = (OFF_BAR + NBAR * 8 + 127) & ~127;
+    static_assert(OFF_MISC % 128 == 0, "control block alignment");
+    static constexpr int MISC_BYTES = 1536 + 4 * (kMaxGrid + 1) + 4 * (kMaxWeightedB + 1);
     static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static constexpr uint32_t TM_COLS = 64;
@@ -154,6 +157,8 @@ struct DecMisc {
     int mslot[kMaxMergeSlots];
     Seg jobs[2];
     int ticket[2];
+    int bounds[kMaxGrid + 1];  // flat start of every CTA's span (cost-weighted), bounds[NC] = tot
+    int yb[kMaxWeightedB + 1]; // weighted start of every batch (the plan's table)
 };
 
 // Reduce NR per-thread values over the 32 lanes of a warp, one row per lane group:
@@ -266,6 +271,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int i = 0; i < C::STV; ++i) ptx::mbar_init(bar(C::B_VCONV + i), 4);
         for (int i = 0; i < C::QBUF; ++i) ptx::mbar_init(bar(C::B_QCONV + i), 4);
         ptx::mbar_init(bar(C::B_OFREE), 4);
+        ptx::mbar_init(bar(C::B_BOUNDS), 1);
         ptx::mbar_init(bar(C::B_RED), 4);
         ptx::mbar_init(bar(C::B_XSYNC), 4);
         ptx::mbar_init(bar(C::B_FINAL), 1);
@@ -280,7 +286,10 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ptx::tmem_alloc(ptx::smem_addr(&misc->tmem_base), C::TM_COLS);
         ptx::tmem_relinquish();
     }
-    if (warp == 0) plan_span(p, cta, NC, &misc->span);
+    if (warp == 0) {
+        if (p.B <= kMaxWeightedB) plan_span_weighted(p, cta, NC, &misc->span, misc->yb);
+        else plan_span(p, cta, NC, &misc->span);  // equal spans (the host sets seg_w = 0)
+    }
     if (warp >= 4 && warp < 8) {
         // P' rows past NR are never written by the softmax: keep them zero
         uint4* pz = reinterpret_cast<uint4*>(smem + C::OFF_P);
@@ -432,19 +441,31 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             drain_bar(bar(C::B_FINAL), 1, p.timeout_cycles);
         }
         // ------------------------------------------------------------ ticket taker
-        else if (warp == 3 && lane == 0) {
+        else if (warp == 3) {
+            // the whole warp fills the span bounds of every CTA (the tickets and the
+            // merges look other CTAs' spans up there), then lane 0 takes the tickets
+            if (p.B <= kMaxWeightedB) {
+                fill_span_bounds(p, misc->yb, NC, misc->bounds);
+            } else {
+                for (int k = lane; k <= NC; k += 32)
+                    misc->bounds[k] = static_cast<int>(span_begin(k, misc->span.tot, NC));
+                __syncwarp();
+            }
+            if (lane == 0) ptx::mbar_arrive(bar(C::B_BOUNDS));
+        }
+        if (warp == 3 && lane == 0) {
             SegWalker wk;
             wk.init(p, misc->span, cta);
             Seg sg;
             int j = 0;
-            const long long tot = misc->span.tot;
             while (j < 2 && wk.next(p, sg)) {
                 if (sg.kind != 1) continue;
                 if (!wait_bar(bar(C::B_MJOB + j), 0, wmisc, p)) break;
-                const int c_first = cta_of(sg.pw, tot, NC);
-                const int c_last = cta_of(sg.pw + sg.ntiles - 1, tot, NC);
+                const int* bd = misc->bounds;
+                const int c_first = cta_of_table(bd, NC, sg.pw);
+                const int c_last = cta_of_table(bd, NC, sg.pw + sg.ntiles - 1);
                 int ncontrib = 0;
-                for (int cc = c_first; cc <= c_last; ++cc) ncontrib += span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC);
+                for (int cc = c_first; cc <= c_last; ++cc) ncontrib += bd[cc] < bd[cc + 1];
                 __threadfence();
                 const int old = atomicAdd(p.counters + sg.w, 1);
                 misc->ticket[j] = (old == ncontrib - 1);
@@ -690,19 +711,21 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             if (!misc->ticket[j]) continue;
+            ok = __all_sync(0xffffffffu, wait_bar(bar(C::B_BOUNDS), 0, wmisc, p));
+            if (!ok) break;
             __threadfence();
             const Seg sgm = misc->jobs[j];
             const RB rb = rb_of(p, sgm.w);
-            const long long tot = misc->span.tot;
-            const int c_first = cta_of(sgm.pw, tot, NC);
-            const int c_last = cta_of(sgm.pw + sgm.ntiles - 1, tot, NC);
-            const bool c0_first = span_begin(c_first, tot, NC) == sgm.pw;
+            const int* bd = misc->bounds;
+            const int c_first = cta_of_table(bd, NC, sgm.pw);
+            const int c_last = cta_of_table(bd, NC, sgm.pw + sgm.ntiles - 1);
+            const bool c0_first = bd[c_first] == sgm.pw;
             const long long RW = BM;
             if (warp == 4) {
                 int nm = 0;
                 for (int base = c_first; base <= c_last; base += 32) {
                     const int cc = base + lane;
-                    const bool has = cc <= c_last && span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC);
+                    const bool has = cc <= c_last && bd[cc] < bd[cc + 1];
                     const unsigned m = __ballot_sync(0xffffffffu, has);
                     const int k = nm + __popc(m & ((1u << lane) - 1u));
                     if (has && k < kMaxMergeSlots) misc->mslot[k] = static_cast<int>(merge_slot(cc, c_first, c0_first));
@@ -716,7 +739,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (nm <= kMaxMergeSlots) return misc->mslot[k];
                 int seen = 0;
                 for (int cc = c_first; cc <= c_last; ++cc) {
-                    if (!(span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC))) continue;
+                    if (!(bd[cc] < bd[cc + 1])) continue;
                     if (seen++ == k) return merge_slot(cc, c_first, c0_first);
                 }
                 return 0;

@@ -68,7 +68,9 @@ struct Fwd2Cfg {
     static constexpr int B_MJOB = B_XSYNC + 1;   // [2] partial rows of split segment j written
     static constexpr int B_MTICK = B_MJOB + 2;   // [2] ticket of split segment j taken
     static constexpr int NBAR = B_MTICK + 2;
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    // the control block holds float4-read arrays: 128-byte aligned whatever NBAR is
+    static constexpr int OFF_MISC = (OFF_BAR + NBAR * 8 + 127) & ~127;
+    static_assert(OFF_MISC % 128 == 0, "control block alignment");
     static constexpr int MISC_BYTES = 2496;
     // the dynamic shared-memory window is required (and checked) to start 1024-aligned
     static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES;

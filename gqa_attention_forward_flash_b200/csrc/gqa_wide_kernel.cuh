@@ -93,6 +93,7 @@ struct WideCfg {
     static constexpr int NBAR = B_MERGE + 1;
     static_assert(NBAR <= 40, "barrier block");
     static constexpr int OFF_MISC = OFF_BAR + 40 * 8;
+    static_assert(OFF_MISC % 16 == 0, "control block alignment");
     static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static constexpr uint32_t TM_COLS = 512;
