@@ -453,6 +453,17 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t issued, long lo
     }
 }
 
+// NaN propagation through the row statistics: a row that met a NaN score or
+// value has a NaN row sum, and its output and log-sum-exp must come out NaN
+// (as IEEE arithmetic on the definition gives), so the maxima below keep NaN
+// (fmaxf would drop it) and a NaN sum takes the branch of a positive one.
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ bool pos_or_nan(float x) { return !(x <= 0.f); }
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -501,9 +512,9 @@ gqa_combine_uniform_kernel(const float* __restrict__ o_part, const float* __rest
         const int h = static_cast<int>((row / Tq) % Hq);
         const float sk = (sink != nullptr) ? sink[h] : -INFINITY;
         float L = sk;
-        for (int s = lane; s < S; s += 32) L = fmaxf(L, lse_part[row * S + s]);
+        for (int s = lane; s < S; s += 32) L = fmax_nan(L, lse_part[row * S + s]);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) L = fmaxf(L, __shfl_xor_sync(0xffffffffu, L, o));
+        for (int o = 16; o > 0; o >>= 1) L = fmax_nan(L, __shfl_xor_sync(0xffffffffu, L, o));
         float lt = -INFINITY;
         if (L != -INFINITY) {
             float z = 0.f;
@@ -562,9 +573,9 @@ gqa_combine_shards_kernel(const __nv_bfloat16* __restrict__ o_sh, long long o_st
         const int h = static_cast<int>((row / Tq) % Hq);
         const float sk = (sink != nullptr) ? sink[h] : -INFINITY;
         float L = sk;
-        for (int s = lane; s < S; s += 32) L = fmaxf(L, l_sh[s * l_stride + row]);
+        for (int s = lane; s < S; s += 32) L = fmax_nan(L, l_sh[s * l_stride + row]);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) L = fmaxf(L, __shfl_xor_sync(0xffffffffu, L, o));
+        for (int o = 16; o > 0; o >>= 1) L = fmax_nan(L, __shfl_xor_sync(0xffffffffu, L, o));
         float lt = -INFINITY;
         if (L != -INFINITY) {
             float z = 0.f;

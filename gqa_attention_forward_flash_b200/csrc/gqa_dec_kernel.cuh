@@ -673,11 +673,11 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (direct) {
                     const int h = rb.g * p.G + r / p.Tq;
                     const float sk = (p.sink != nullptr) ? __ldg(p.sink + h) * LOG2E : -INFINITY;
-                    const float M = fmaxf(em[r], sk);
+                    const float M = fmax_nan(em[r], sk);
                     if (M != -INFINITY) {
-                        const float a = (el[r] > 0.f) ? ptx::ex2(em[r] - M) : 0.f;
+                        const float a = pos_or_nan(el[r]) ? ptx::ex2(em[r] - M) : 0.f;
                         const float lt = el[r] * a + ((sk != -INFINITY) ? ptx::ex2(sk - M) : 0.f);
-                        if (lt > 0.f) {
+                        if (pos_or_nan(lt)) {
                             w = a / lt * p.v_scale;
                             lse_v = (M + __log2f(lt)) * LN2;
                         }
@@ -685,7 +685,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     p.out[fr * C::D + kl] = __float2bfloat16_rn(w != 0.f ? eo[r] * w : 0.f);
                     if (kl == 0 && p.lse != nullptr) p.lse[fr] = lse_v;
                 } else {
-                    if (el[r] > 0.f) {
+                    if (pos_or_nan(el[r])) {
                         w = p.v_scale / el[r];
                         lse_v = (em[r] + __log2f(el[r])) * LN2;
                     }
@@ -756,7 +756,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         lv[jj] = (k0 + jj < nm) ? __ldcg(p.part_lse + slot_of(k0 + jj) * RW + r) : -INFINITY;
                     float mx = Lx;
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) mx = fmaxf(mx, lv[jj]);
+                    for (int jj = 0; jj < 8; ++jj) mx = fmax_nan(mx, lv[jj]);
                     if (mx != -INFINITY) {
                         // running (max, sum) over the pieces seen so far
                         z = (Lx != -INFINITY) ? z * __expf(Lx - mx) : 0.f;

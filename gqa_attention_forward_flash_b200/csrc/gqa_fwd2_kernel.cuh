@@ -100,6 +100,47 @@ struct Misc2 {
     int ticket[2];            // 1: this CTA wrote the row-block's last piece and merges it
 };
 
+// Part of the softmax exponentials run on the FMA pipe instead of the MUFU unit,
+// which computes 16 exp2 per clock per SM: exactly the rate at which the tensor
+// pipe consumes a 128 x 128 score tile, so with every exp2 there the two lanes'
+// softmaxes are the critical path.  Cody and Waite's range reduction: x = n + f
+// with n = round(x) (the 1.5 * 2^23 addition leaves n in the low mantissa bits)
+// and f in [-1/2, 1/2]; 2^f by a cubic whose constant term is exactly 1 and whose
+// other coefficients minimise the largest relative error on [-1/2, 1/2] (a
+// linear program over a fine grid: 1.0e-4, far below the 2^-9 of P's bf16
+// rounding); n is added to the exponent field.  x is clamped to -127 first:
+// there f = 0, the cubic gives exactly 1.0 and the sum of the fields is +0, so a
+// masked score (-inf) still gives an exact 0, and nothing below wraps the field.
+// A NaN x gives 0 here, not NaN: rows whose tile maximum is NaN or +inf carry
+// a NaN row sum instead (see the softmax).
+constexpr float kExp2C1 = 0.693282902f;
+constexpr float kExp2C2 = 0.242210969f;
+constexpr float kExp2C3 = 0.0550090596f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+__device__ __forceinline__ uint64_t exp2_poly_pair(uint64_t x2) {
+    float x0, x1;
+    ptx::f2_split(x2, x0, x1);
+    const uint64_t xc = ptx::f2(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+    const uint64_t mg = ptx::f2(kRoundMagic, kRoundMagic);
+    const uint64_t j = ptx::f2_add(xc, mg);
+    const uint64_t f = ptx::f2_sub(xc, ptx::f2_sub(j, mg));
+    uint64_t q = ptx::f2_fma(ptx::f2(kExp2C3, kExp2C3), f, ptx::f2(kExp2C2, kExp2C2));
+    q = ptx::f2_fma(q, f, ptx::f2(kExp2C1, kExp2C1));
+    q = ptx::f2_fma(q, f, ptx::f2(1.f, 1.f));
+    float j0, j1, q0, q1;
+    ptx::f2_split(j, j0, j1);
+    ptx::f2_split(q, q0, q1);
+    // the low bits of j are n + 2^22; shifted by 23 only n survives
+    const uint32_t r0 = __float_as_uint(q0) + (__float_as_uint(j0) << 23);
+    const uint32_t r1 = __float_as_uint(q1) + (__float_as_uint(j1) << 23);
+    return ptx::f2(__uint_as_float(r0), __uint_as_float(r1));
+}
+// Which of the 16 column pairs of each 32-column chunk take the cubic (bit j).
+#ifndef GQA_POLY_PAIRS
+#define GQA_POLY_PAIRS 0x0u
+#endif
+constexpr uint32_t kPolyPairs = GQA_POLY_PAIRS;
+
 // Load key tile t of row-block rb (n = its batch's logical length) from K or V
 // into one ring stage and arm the stage's full barrier.  Contiguous K/V: one box
 // per 64 columns at row rb.kv_row0 + t*BN of the [B*Hkv*Tkv, d] view.  Paged K/V
@@ -354,10 +395,14 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int t = sg.t0; t < sg.t1 && ok; ++t, ++g) {
                     const int stk = g % C::STK;
                     const int stv = g % C::STV;
-                    ok = wait_bar(bar(C::B_KFULL + stk), (g / C::STK) & 1, wmisc, p);
-                    if (!ok) break;
-                    ptx::tc_fence_after();
                     const uint32_t kbase = sbase + C::OFF_K + stk * C::KV_BYTES;
+                    // dual-Q: S0 of every tile but a segment's first went out at the end of
+                    // the previous iteration, its K stage awaited there
+                    if (C::RBQ == 1 || t == sg.t0) {
+                        ok = wait_bar(bar(C::B_KFULL + stk), (g / C::STK) & 1, wmisc, p);
+                        if (!ok) break;
+                        ptx::tc_fence_after();
+                    }
                     if (C::RBQ == 1) {
                         const int L = g & 1;
                         issue_s(L, qbase, kbase);
@@ -374,7 +419,11 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         prev_first = !lane_seen[L];
                         lane_seen[L] = true;
                     } else {
-                        issue_s(0, qbase, kbase);
+                        // A wait in this thread stalls the tensor pipe for about 130 cycles
+                        // even on a completed barrier, so lane 0's chain (P0 -> PV0 -> next
+                        // S0 -> softmax) keeps one wait, on P0: V(t) and K(t+1) are awaited
+                        // while S1(t) executes.
+                        if (t == sg.t0) issue_s(0, qbase, kbase);
                         if (have_b) {
                             ok = issue_pv(1, b_stv, b_first, false, 0);
                             if (!ok) break;
@@ -383,8 +432,17 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         issue_s(1, qbase + C::Q_TILE, kbase);
                         ptx::umma_commit(bar(C::B_KEMPTY + stk));
                         if (t == sg.t1 - 1) ptx::umma_commit(bar(C::B_QEMPTY));
-                        ok = issue_pv(0, stv, t == sg.t0, true, g);
+                        ok = wait_bar(bar(C::B_VFULL + stv), (g / C::STV) & 1, wmisc, p);
                         if (!ok) break;
+                        const bool more = t + 1 < sg.t1;
+                        const int stk1 = (g + 1) % C::STK;
+                        if (more) {
+                            ok = wait_bar(bar(C::B_KFULL + stk1), ((g + 1) / C::STK) & 1, wmisc, p);
+                            if (!ok) break;
+                        }
+                        ok = issue_pv(0, stv, t == sg.t0, false, g);
+                        if (!ok) break;
+                        if (more) issue_s(0, qbase, sbase + C::OFF_K + stk1 * C::KV_BYTES);
                         have_b = true;
                         b_first = (t == sg.t0);
                         b_stv = stv;
@@ -510,15 +568,16 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                         for (int c = 0; c < C::BN; ++c) s[c] = (c <= lim) ? s[c] : -INFINITY;
                     }
+                    // the tile maximum; NaN if any visible score is NaN
                     float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                    for (int c = 0; c < C::BN; c += 4) {
-                        m4[0] = fmaxf(m4[0], s[c]);
-                        m4[1] = fmaxf(m4[1], s[c + 1]);
-                        m4[2] = fmaxf(m4[2], s[c + 2]);
-                        m4[3] = fmaxf(m4[3], s[c + 3]);
+                    for (int c = 0; c < C::BN; c += 8) {
+                        m4[0] = ptx::max3_nan(m4[0], s[c], s[c + 1]);
+                        m4[1] = ptx::max3_nan(m4[1], s[c + 2], s[c + 3]);
+                        m4[2] = ptx::max3_nan(m4[2], s[c + 4], s[c + 5]);
+                        m4[3] = ptx::max3_nan(m4[3], s[c + 6], s[c + 7]);
                     }
-                    const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.scale_log2;
+                    const float mt = ptx::max3_nan(m4[0], m4[1], ptx::max3_nan(m4[2], m4[3], m4[3])) * p.scale_log2;
                     if (first) {
                         m_ref = mt;
                     } else if (mt > m_ref + RESCALE_THRESHOLD) {
@@ -528,21 +587,37 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     // P = 2^(s*scale*log2e - m) as bf16 over the lane's S columns [64, 128)
                     const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
                     const uint32_t tp = tmem + lane_off + C::tm_p(L);
-                    float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+                    const uint64_t sl2 = ptx::f2(p.scale_log2, p.scale_log2);
+                    const uint64_t nm2 = ptx::f2(neg_m, neg_m);
+                    uint64_t acc[4];
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) acc[a] = ptx::f2(0.f, 0.f);
 #pragma unroll
                     for (int c = 0; c < C::BN / 32; ++c) {
                         uint32_t pk[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            const float a = ptx::ex2(fmaf(s[c * 32 + 2 * j], p.scale_log2, neg_m));
-                            const float b = ptx::ex2(fmaf(s[c * 32 + 2 * j + 1], p.scale_log2, neg_m));
-                            rs4[(2 * j) & 3] += a;
-                            rs4[(2 * j + 1) & 3] += b;
-                            pk[j] = pack_bf16x2(a, b);
+                            const uint64_t x2 = ptx::f2_fma(ptx::f2(s[c * 32 + 2 * j], s[c * 32 + 2 * j + 1]), sl2, nm2);
+                            uint64_t e2;
+                            if ((kPolyPairs >> j) & 1u) {
+                                e2 = exp2_poly_pair(x2);
+                            } else {
+                                float x0, x1;
+                                ptx::f2_split(x2, x0, x1);
+                                e2 = ptx::f2(ptx::ex2(x0), ptx::ex2(x1));
+                            }
+                            acc[j & 3] = ptx::f2_add(acc[j & 3], e2);
+                            float e0, e1;
+                            ptx::f2_split(e2, e0, e1);
+                            pk[j] = pack_bf16x2(e0, e1);
                         }
                         ptx::tmem_st16(tp + c * 16, pk);
                     }
-                    l_sum = l_sum * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
+                    float a0, a1;
+                    ptx::f2_split(ptx::f2_add(ptx::f2_add(acc[0], acc[1]), ptx::f2_add(acc[2], acc[3])), a0, a1);
+                    l_sum = l_sum * alpha + (a0 + a1);
+                    // a NaN or +inf maximum: the cubic turned NaN scores into 0, so mark the row
+                    if (mt != mt || mt == INFINITY) l_sum = __int_as_float(0x7fffffff);
                 }
                 // lazy rescale of the lane's O: only when a row's max grew by more than 2^8
                 if (!first && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -611,12 +686,12 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const float mo = misc->st_m[L ^ 1][lrow], lo = misc->st_l[L ^ 1][lrow];
                 const float mm = (mine > 0) ? m_ref : -INFINITY, ll = (mine > 0) ? l_sum : 0.f;
                 const float sk = (direct && p.sink != nullptr && valid) ? __ldg(p.sink + h) * LOG2E : -INFINITY;
-                const float M = fmaxf(fmaxf(mm, mo), sk);
+                const float M = fmax_nan(fmax_nan(mm, mo), sk);
                 if (M != -INFINITY) {
-                    const float a = (ll > 0.f) ? ptx::ex2(mm - M) : 0.f;
-                    const float b = (lo > 0.f) ? ptx::ex2(mo - M) : 0.f;
+                    const float a = pos_or_nan(ll) ? ptx::ex2(mm - M) : 0.f;
+                    const float b = pos_or_nan(lo) ? ptx::ex2(mo - M) : 0.f;
                     const float lt = ll * a + lo * b + ((sk != -INFINITY) ? ptx::ex2(sk - M) : 0.f);
-                    if (lt > 0.f) {
+                    if (pos_or_nan(lt)) {
                         w_own = a / lt;
                         w_oth = b / lt;
                         lse_v = (M + __log2f(lt)) * LN2;
@@ -624,11 +699,11 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             } else {
                 const float sk = (direct && p.sink != nullptr && valid) ? __ldg(p.sink + h) * LOG2E : -INFINITY;
-                const float M = fmaxf(m_ref, sk);
+                const float M = fmax_nan(m_ref, sk);
                 if (M != -INFINITY) {
-                    const float a = (l_sum > 0.f) ? ptx::ex2(m_ref - M) : 0.f;
+                    const float a = pos_or_nan(l_sum) ? ptx::ex2(m_ref - M) : 0.f;
                     const float lt = l_sum * a + ((sk != -INFINITY) ? ptx::ex2(sk - M) : 0.f);
-                    if (lt > 0.f) {
+                    if (pos_or_nan(lt)) {
                         w_own = a / lt;
                         lse_v = (M + __log2f(lt)) * LN2;
                     }
@@ -741,7 +816,7 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             for (int j = 0; j < 8; ++j)
                                 lv[j] = (k0 + j < nm) ? __ldcg(p.part_lse + misc->mslot[k0 + j] * RW + r) : -INFINITY;
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) Lx = fmaxf(Lx, lv[j]);
+                            for (int j = 0; j < 8; ++j) Lx = fmax_nan(Lx, lv[j]);
                         }
                         float lt = -INFINITY;
                         if (Lx != -INFINITY) {
@@ -800,7 +875,7 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         float Lx = (p.sink != nullptr) ? __ldg(p.sink + hr) : -INFINITY;
                         for (int cc = c_first; cc <= c_last; ++cc) {
                             if (!(span_begin(cc, tot, NC) < span_begin(cc + 1, tot, NC))) continue;
-                            Lx = fmaxf(Lx, __ldcg(p.part_lse + merge_slot(cc, c_first, c0_first) * RW + r));
+                            Lx = fmax_nan(Lx, __ldcg(p.part_lse + merge_slot(cc, c_first, c0_first) * RW + r));
                         }
                         float lt = -INFINITY;
                         if (Lx != -INFINITY) {

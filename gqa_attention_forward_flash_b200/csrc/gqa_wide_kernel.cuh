@@ -532,16 +532,16 @@ gqa_wide_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (nonempty) {
                 if (sg.kind == 0) {
                     const float sk = (p.sink != nullptr && valid) ? __ldg(p.sink + h) * LOG2E : -INFINITY;
-                    const float M = fmaxf(m_ref, sk);
+                    const float M = fmax_nan(m_ref, sk);
                     if (M != -INFINITY) {
-                        const float a = (l_sum > 0.f) ? ptx::ex2(m_ref - M) : 0.f;
+                        const float a = pos_or_nan(l_sum) ? ptx::ex2(m_ref - M) : 0.f;
                         const float lt = l_sum * a + ((sk != -INFINITY) ? ptx::ex2(sk - M) : 0.f);
-                        if (lt > 0.f) {
+                        if (pos_or_nan(lt)) {
                             o_scale = a / lt;
                             lse_v = (M + __log2f(lt)) * LN2;
                         }
                     }
-                } else if (l_sum > 0.f) {
+                } else if (pos_or_nan(l_sum)) {
                     o_scale = 1.f / l_sum;
                     lse_v = (m_ref + __log2f(l_sum)) * LN2;
                 }
@@ -707,13 +707,13 @@ gqa_wide_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         // lse of this thread's row over the pieces (the sink enters once,
                         // here), then the pieces' weights in place of their lse
                         float mx = sk;
-                        for (int k = 0; k < nc; ++k) mx = fmaxf(mx, lse_st[k * BM + r]);
+                        for (int k = 0; k < nc; ++k) mx = fmax_nan(mx, lse_st[k * BM + r]);
                         float z = 0.f;
                         if (mx != -INFINITY) {
                             for (int k = 0; k < nc; ++k) z += __expf(lse_st[k * BM + r] - mx);
                             if (sk != -INFINITY) z += __expf(sk - mx);
                         }
-                        const float lt = (mx != -INFINITY && z > 0.f) ? mx + __logf(z) : -INFINITY;
+                        const float lt = (mx != -INFINITY && pos_or_nan(z)) ? mx + __logf(z) : -INFINITY;
                         for (int k = 0; k < nc; ++k)
                             lse_st[k * BM + r] = (lt != -INFINITY) ? __expf(lse_st[k * BM + r] - lt) : 0.f;
                         if (kme == 0 && ho == 0 && r < rows && p.lse != nullptr) p.lse[rb.q_row0 + r] = lt;
@@ -753,13 +753,13 @@ gqa_wide_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     return 0;
                 };
                 float mx = sk;
-                for (int k = 0; k < nc; ++k) mx = fmaxf(mx, __ldcg(p.part_lse + slot_of(k) * BM + r));
+                for (int k = 0; k < nc; ++k) mx = fmax_nan(mx, __ldcg(p.part_lse + slot_of(k) * BM + r));
                 float z = 0.f;
                 if (mx != -INFINITY) {
                     for (int k = 0; k < nc; ++k) z += __expf(__ldcg(p.part_lse + slot_of(k) * BM + r) - mx);
                     if (sk != -INFINITY) z += __expf(sk - mx);
                 }
-                const float lt = (mx != -INFINITY && z > 0.f) ? mx + __logf(z) : -INFINITY;
+                const float lt = (mx != -INFINITY && pos_or_nan(z)) ? mx + __logf(z) : -INFINITY;
                 if (kme == 0 && ho == 0 && r < rows && p.lse != nullptr) p.lse[rb.q_row0 + r] = lt;
                 if (r < rows) {
                     __nv_bfloat16* orow = p.out + (rb.q_row0 + r) * C::D + ho * C::DO;

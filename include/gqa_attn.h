@@ -18,7 +18,11 @@
  *           domain: it is never multiplied by `scale` (dsv4 attention commit
  *           log, sink commit)
  *     lse[b,h,i] = ln( sum_visible exp(s_j) + exp(sink[h]) ), natural log
- *   A row with no visible key and no sink gets O = 0 and lse = -inf.  The
+ *   A row with no visible key and no sink gets O = 0 and lse = -inf.  A NaN
+ *   or inf inside the first n rows of K or V makes the rows that see it NaN
+ *   (IEEE arithmetic on the definition); a V value of that kind also reaches
+ *   the rows of its 128-key tile that mask it by causality (their weight 0
+ *   times NaN), so K/V should be finite inside the logical lengths.  The
  *   computation is tile by tile with an online-softmax (m, l, O) carry (dsv4
  *   attention commit log, multi-tile commit: running max/sum rescale, O / l
  *   once at the end); long key ranges are split over SMs and the partial

@@ -152,7 +152,8 @@ def _two_lane(segs, rbq, stk, stv, rnd, mutate=False):
             prev = None
             pend_b = None
             for t in range(n):
-                yield ("wait", "KF%d" % (g % stk), g // stk)
+                if rbq == 1 or t == 0:
+                    yield ("wait", "KF%d" % (g % stk), g // stk)
                 last = ["QEMPTY"] if t == n - 1 else []
                 if rbq == 1:
                     lane = g & 1
@@ -161,11 +162,18 @@ def _two_lane(segs, rbq, stk, stv, rnd, mutate=False):
                         yield from pv(prev[0], prev[1], True)
                     prev = (lane, g)
                 else:
-                    yield ("mma", ["SF0"])
+                    if t == 0:
+                        yield ("mma", ["SF0"])
                     if pend_b is not None:
                         yield from pv(1, pend_b, False)
                     yield ("mma", ["SF1", "KE%d" % (g % stk)] + last)
-                    yield from pv(0, g, True)
+                    # V(t) and K(t+1) awaited before P0(t); S0(t+1) right after PV0(t)
+                    yield ("wait", "VF%d" % (g % stv), g // stv)
+                    if t + 1 < n:
+                        yield ("wait", "KF%d" % ((g + 1) % stk), (g + 1) // stk)
+                    yield from pv(0, g, False)
+                    if t + 1 < n:
+                        yield ("mma", ["SF0"])
                     pend_b = g
                 g += 1
             # the segment's last PV goes out when its tile loop ends
