@@ -16,14 +16,19 @@
 // 128-byte swizzle) goes to shared memory as the B operand of the second MMA;
 // V's shared-memory tile serves as the MN-major A operand V^T unchanged.
 //
-//   TMEM columns  [0,16) S'0   [16,32) S'1   [32,48) O'
+//   TMEM columns  [0,16) S'0   [16,32) S'1   [32,48) O'0   [48,64) O'1
 //
 // MMA order (one thread): S'(g), PV'(g-1), S'(g+1), PV'(g), ...  S' is double
-// buffered; P' is double buffered; the softmax of tile g overlaps PV'(g-1).
+// buffered; P' is double buffered; the softmax of tile g overlaps PV'(g-1).  O'
+// is double buffered by segment (segment s accumulates in O'(s % 2)), so that the
+// softmax goes on with the next segment while segment s is finished: its row
+// statistics go to shared memory, and an epilogue warpgroup (warps 8-11, warp
+// 8+q reading TMEM lane quadrant q) writes the output rows or the split piece,
+// takes the piece's ticket and merges the row-block if the piece completes it.
 // Warps: 0 Q/K producer (and the stream-K plan), 1 V producer, 2 TMEM owner +
-// MMA issuer, 3 split-segment ticket taker, 4-7 softmax (warp 4+q reads TMEM
-// lane quadrant q).  The stream-K work split, the split partial slots and the
-// last-arriver merge are those of the two-lane kernel (gqa_fwd2_kernel.cuh).
+// MMA issuer, 3 span-bounds table, 4-7 softmax (warp 4+q reads TMEM lane
+// quadrant q), 8-11 epilogue.  The stream-K work split, the split partial slots
+// and the last-arriver merge are those of the two-lane kernel (gqa_fwd2_kernel.cuh).
 //
 // FP8 K/V (FP8 = true; the AstrAI commit log's fp8 family stores tensors as E4M3
 // with one scale per tensor): each K/V tile arrives by TMA as 128 keys x 128
@@ -32,7 +37,8 @@
 // zeroing V rows past the logical length as they go; Q is converted from bf16
 // to f16 in place once per segment, and P' is written as f16, so both MMAs run
 // with f16 operands.  k_scale is folded into the logit scale and v_scale into
-// the output normalisation.
+// the output normalisation.  With the converter warps in warps 8-11, the softmax
+// warps run each segment's epilogue themselves (the same code, same barriers).
 #pragma once
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -41,7 +47,6 @@
 
 namespace gqa {
 
-constexpr int NUM_THREADS_DEC = 256;
 constexpr int NSOFT_DEC = 128;
 constexpr int DEC_NQ = 16;  // N of both MMAs: packed query rows held (padded)
 
@@ -53,7 +58,8 @@ struct DecCfg {
     static constexpr bool PAGED = PAGED_;
     static constexpr bool FP8 = FP8_;  // K/V stored as E4M3 bytes (contiguous caches only)
     static_assert(!(PAGED && FP8), "fp8 K/V over a paged cache is not built");
-    static constexpr int NTHREADS = FP8 ? 384 : 256;  // + four converter warps
+    static constexpr int NTHREADS = 384;  // + four epilogue warps (bf16) or converter warps (FP8)
+    static constexpr bool EPIW = !FP8;    // a separate epilogue warpgroup runs the segment epilogues
     static constexpr int NBOX = D / 64;
     static constexpr int KV_BOX = BN * 128;             // one 64-column box of a K/V tile
     static constexpr int KV_BYTES = NBOX * KV_BOX;
@@ -75,13 +81,14 @@ struct DecCfg {
     static constexpr int B_SFULL = B_VEMPTY + STV;      // [2] S' buffer written
     static constexpr int B_PFULL = B_SFULL + 2;         // [2] P' buffer written (one arrival per softmax warp)
     static constexpr int B_PVDONE = B_PFULL + 2;        // [2] PV' that read P' buffer b completed
-    static constexpr int B_OFREE = B_PVDONE + 2;        // segment epilogue has read O'
-    static constexpr int B_RED = B_OFREE + 1;           // softmax warps: per-tile row reductions
-    static constexpr int B_XSYNC = B_RED + 1;           // softmax warps: epilogue / merge steps
-    static constexpr int B_FINAL = B_XSYNC + 1;
-    static constexpr int B_MJOB = B_FINAL + 1;          // [2] partial rows of split segment j written
-    static constexpr int B_MTICK = B_MJOB + 2;          // [2] ticket of split segment j taken
-    static constexpr int B_KCONV = B_MTICK + 2;         // [STK] FP8: K stage widened to f16
+    static constexpr int B_OFREE = B_PVDONE + 2;        // [2] epilogue has read O' buffer b and its row stats
+    static constexpr int B_STATS = B_OFREE + 2;         // [2] softmax has written the row stats of buffer b
+    static constexpr int B_SEGPV = B_STATS + 2;         // [2] a segment's last PV' into O' buffer b completed
+    static constexpr int B_RED = B_SEGPV + 2;           // softmax warps: per-tile row reductions
+    static constexpr int B_XSYNC = B_RED + 1;           // softmax warps: epilogue / merge steps (FP8)
+    static constexpr int B_ESYNC = B_XSYNC + 1;         // epilogue warps: epilogue / merge steps
+    static constexpr int B_FINAL = B_ESYNC + 1;
+    static constexpr int B_KCONV = B_FINAL + 1;         // [STK] FP8: K stage widened to f16
     static constexpr int B_VCONV = B_KCONV + STK;       // [STV] FP8: V stage widened to f16
     static constexpr int B_QCONV = B_VCONV + STV;       // [QBUF] FP8: Q buffer converted to f16
     static constexpr int B_BOUNDS = B_QCONV + QBUF;     // the span bounds table is filled
@@ -94,7 +101,7 @@ struct DecCfg {
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static constexpr uint32_t TM_COLS = 64;
     static constexpr uint32_t TM_S = 0;   // + 16 * buffer
-    static constexpr uint32_t TM_O = 32;
+    __host__ __device__ static constexpr uint32_t tm_o(int b) { return 32u + 16u * static_cast<uint32_t>(b); }
     static constexpr uint32_t IDESC_S =
         FP8 ? ptx::umma_idesc_f16_f32(BN, DEC_NQ, false, false) : ptx::umma_idesc_bf16_f32(BN, DEC_NQ, false, false);
     static constexpr uint32_t IDESC_PV =
@@ -155,8 +162,9 @@ struct DecMisc {
     float mlse[DEC_NQ];       // merged lse per packed row (in-kernel merge)
     int nmerge;
     int mslot[kMaxMergeSlots];
-    Seg jobs[2];
-    int ticket[2];
+    float seg_w[2][DEC_NQ];   // per row of the segment in O' buffer b: the factor O' is scaled by
+    float seg_lse[2][DEC_NQ]; //   and the row's (or the piece's) lse
+    int etk;                  // the epilogue's split piece completed its row-block (it merges)
     int bounds[kMaxGrid + 1];  // flat start of every CTA's span (cost-weighted), bounds[NC] = tot
     int yb[kMaxWeightedB + 1]; // weighted start of every batch (the plan's table)
 };
@@ -204,12 +212,14 @@ __device__ __forceinline__ bool dec_row_writer(int lane) {
 // runs at a segment switch would be fetched while every SM streams K/V).
 template <class C>
 __device__ __noinline__ bool dec_issue_pv(const Params& p, Misc* wmisc, uint32_t bar0, uint32_t sbase, uint32_t tmem,
-                                          uint32_t gg, bool first, int seg) {
+                                          uint32_t gg, bool first, int seg, bool last) {
     auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
     const int st = gg % C::STV;
+    const int ob = seg & 1;
     if (!wait_bar(bar(C::B_PFULL + (gg & 1u)), (gg >> 1) & 1u, wmisc, p)) return false;
     if (!wait_bar(bar(C::B_VREADY + st), (gg / C::STV) & 1u, wmisc, p)) return false;
-    if (first && seg > 0 && !wait_bar(bar(C::B_OFREE), (seg - 1) & 1, wmisc, p)) return false;
+    // a segment's first PV' overwrites O' buffer seg % 2: its epilogue two segments back must have read it
+    if (first && seg >= 2 && !wait_bar(bar(C::B_OFREE + ob), ((seg - 2) >> 1) & 1, wmisc, p)) return false;
     ptx::tc_fence_after();
     const uint32_t vbase = sbase + C::OFF_V + st * C::KV_BYTES;
     const uint32_t pbase = sbase + C::OFF_P + (gg & 1u) * C::P_BYTES;
@@ -217,10 +227,11 @@ __device__ __noinline__ bool dec_issue_pv(const Params& p, Misc* wmisc, uint32_t
     for (int kk = 0; kk < C::BN / 16; ++kk) {
         const uint64_t ad = ptx::umma_desc_sw128(vbase + kk * 2048, C::KV_BOX, 1024);
         const uint64_t bd = ptx::umma_desc_sw128(pbase + (kk >> 2) * C::P_BOX + (kk & 3) * 32, 16, 1024);
-        ptx::umma_bf16_ss(tmem + C::TM_O, ad, bd, C::IDESC_PV, (kk > 0 || !first) ? 1u : 0u);
+        ptx::umma_bf16_ss(tmem + C::tm_o(ob), ad, bd, C::IDESC_PV, (kk > 0 || !first) ? 1u : 0u);
     }
     ptx::umma_commit(bar(C::B_PVDONE + (gg & 1u)));
     ptx::umma_commit(bar(C::B_VEMPTY + st));
+    if (last) ptx::umma_commit(bar(C::B_SEGPV + ob));
     return true;
 }
 
@@ -264,16 +275,17 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ptx::mbar_init(bar(C::B_SFULL + i), 1);
             ptx::mbar_init(bar(C::B_PFULL + i), 4);
             ptx::mbar_init(bar(C::B_PVDONE + i), 1);
-            ptx::mbar_init(bar(C::B_MJOB + i), 1);
-            ptx::mbar_init(bar(C::B_MTICK + i), 1);
+            ptx::mbar_init(bar(C::B_OFREE + i), 4);  // one arrival per epilogue warp
+            ptx::mbar_init(bar(C::B_STATS + i), 4);  // one arrival per softmax warp
+            ptx::mbar_init(bar(C::B_SEGPV + i), 1);
         }
         for (int i = 0; i < C::STK; ++i) ptx::mbar_init(bar(C::B_KCONV + i), 4);
         for (int i = 0; i < C::STV; ++i) ptx::mbar_init(bar(C::B_VCONV + i), 4);
         for (int i = 0; i < C::QBUF; ++i) ptx::mbar_init(bar(C::B_QCONV + i), 4);
-        ptx::mbar_init(bar(C::B_OFREE), 4);
         ptx::mbar_init(bar(C::B_BOUNDS), 1);
         ptx::mbar_init(bar(C::B_RED), 4);
         ptx::mbar_init(bar(C::B_XSYNC), 4);
+        ptx::mbar_init(bar(C::B_ESYNC), 4);
         ptx::mbar_init(bar(C::B_FINAL), 1);
         misc->abort = 0;
         misc->merge_flag = 0;
@@ -301,6 +313,174 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = misc->tmem_base;
+
+    // The epilogue of segment seg_i, by four warps (warp q reads TMEM lane
+    // quadrant q; thread et = 32q + lane owns head dim et): O'(seg_i % 2) times
+    // 1/l written as the output rows (a direct segment) or as a split piece; a
+    // piece then takes the row-block's ticket, and the piece that completes the
+    // row-block merges all of its pieces.  `sync` is the four warps' bounded
+    // barrier.  The row loops are rolled: this code first runs while every SM
+    // streams K/V, and each of its instruction-cache lines is fetched then.
+    auto epi_segment = [&](const Seg& sg, int seg_i, int q, auto&& sync) -> bool {
+        const int ob = seg_i & 1;
+        const int et = q * 32 + lane;
+        const int kl = et;
+        const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+        bool ok = __all_sync(0xffffffffu, wait_bar(bar(C::B_STATS + ob), (seg_i >> 1) & 1, wmisc, p));
+        if (ok) ok = __all_sync(0xffffffffu, wait_bar(bar(C::B_SEGPV + ob), (seg_i >> 1) & 1, wmisc, p));
+        if (!ok) return false;
+        ptx::tc_fence_after();
+        const RB rb = rb_of(p, sg.w);
+        uint32_t o[NR];
+        {
+            const uint32_t to = tmem + lane_off + C::tm_o(ob);
+            if constexpr (NR == 16) ptx::tmem_ld16(to, o);
+            else ptx::tmem_ld8(to, o);
+            ptx::tmem_wait_ld();
+        }
+        float w[NR], lse_r[NR];
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+            w[r] = misc->seg_w[ob][r];
+            lse_r[r] = misc->seg_lse[ob][r];
+        }
+        // O'(ob) and the row factors are read: the segment after next may use them
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(C::B_OFREE + ob));
+        const bool direct = (sg.kind == 0);
+        if (direct) {
+#pragma unroll
+            for (int r = 0; r < NR; ++r)
+                if (r < rb.rows_valid) {
+                    const long long fr = rb.q_row0 + r;  // flat row (b*Hq + h)*Tq + i
+                    p.out[fr * C::D + kl] = __float2bfloat16_rn(w[r] != 0.f ? __uint_as_float(o[r]) * w[r] : 0.f);
+                    if (kl == 0 && p.lse != nullptr) p.lse[fr] = lse_r[r];
+                }
+        } else {
+#pragma unroll
+            for (int r = 0; r < NR; ++r)
+                if (r < rb.rows_valid) {
+                    const long long prow = static_cast<long long>(sg.slot) * BM + r;
+                    __stcg(p.part_o + prow * C::D + kl, w[r] != 0.f ? __uint_as_float(o[r]) * w[r] : 0.f);
+                    if (kl == 0) __stcg(p.part_lse + prow, lse_r[r]);
+                }
+            // release: this thread's partial rows are visible GPU-wide before the ticket
+            __threadfence();
+        }
+        if (direct) return true;
+        // a split piece: once all of its rows are written, count it on the
+        // row-block's ticket (release fence, then the atomic)
+        if (!sync()) return false;
+        if (et == 0) {
+            int tk = 0;
+            if (wait_bar(bar(C::B_BOUNDS), 0, wmisc, p)) {
+                const int* bd = misc->bounds;
+                const int c_first = cta_of_table(bd, NC, sg.pw);
+                const int c_last = cta_of_table(bd, NC, sg.pw + sg.ntiles - 1);
+                int ncontrib = 0;
+                for (int cc = c_first; cc <= c_last; ++cc) ncontrib += bd[cc] < bd[cc + 1];
+                const int old = atomicAdd(p.counters + sg.w, 1);
+                tk = (old == ncontrib - 1);
+            }
+            misc->etk = tk;
+        }
+        if (!sync() || misc->abort) return false;
+        if (!misc->etk) return true;
+        // this piece completed the row-block: merge every piece's rows
+        __threadfence();
+        const int* bd = misc->bounds;
+        const int c_first = cta_of_table(bd, NC, sg.pw);
+        const int c_last = cta_of_table(bd, NC, sg.pw + sg.ntiles - 1);
+        const bool c0_first = bd[c_first] == sg.pw;
+        const long long RW = BM;
+        if (q == 0) {
+            int nm = 0;
+            for (int base = c_first; base <= c_last; base += 32) {
+                const int cc = base + lane;
+                const bool has = cc <= c_last && bd[cc] < bd[cc + 1];
+                const unsigned m = __ballot_sync(0xffffffffu, has);
+                const int k = nm + __popc(m & ((1u << lane) - 1u));
+                if (has && k < kMaxMergeSlots) misc->mslot[k] = static_cast<int>(merge_slot(cc, c_first, c0_first));
+                nm += __popc(m);
+            }
+            if (lane == 0) misc->nmerge = nm;
+        }
+        if (!sync()) return false;
+        const int nm = misc->nmerge;
+        auto slot_of = [&](int k) -> long long {  // k-th contributing CTA's slot
+            if (nm <= kMaxMergeSlots) return misc->mslot[k];
+            int seen = 0;
+            for (int cc = c_first; cc <= c_last; ++cc) {
+                if (!(bd[cc] < bd[cc + 1])) continue;
+                if (seen++ == k) return merge_slot(cc, c_first, c0_first);
+            }
+            return 0;
+        };
+        // lse of each merged row (the sink enters here, once); eight pieces' loads at a time
+        for (int r = et; r < rb.rows_valid; r += 128) {
+            const int hr = rb.g * p.G + r / p.Tq;
+            const float sk = (p.sink != nullptr) ? __ldg(p.sink + hr) : -INFINITY;
+            float Lx = sk, z = 0.f;
+            for (int k0 = 0; k0 < nm; k0 += 8) {
+                float lv[8];
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj)
+                    lv[jj] = (k0 + jj < nm) ? __ldcg(p.part_lse + slot_of(k0 + jj) * RW + r) : -INFINITY;
+                float mx = Lx;
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) mx = fmax_nan(mx, lv[jj]);
+                if (mx != -INFINITY) {
+                    // running (max, sum) over the pieces seen so far
+                    z = (Lx != -INFINITY) ? z * __expf(Lx - mx) : 0.f;
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) z += __expf(lv[jj] - mx);
+                    Lx = mx;
+                }
+            }
+            float ltr = -INFINITY;
+            if (Lx != -INFINITY) {
+                if (sk != -INFINITY) z += __expf(sk - Lx);
+                ltr = Lx + __logf(z);
+            }
+            misc->mlse[r] = ltr;
+            if (p.lse != nullptr) p.lse[rb.q_row0 + r] = ltr;
+        }
+        if (!sync()) return false;
+        // O rows: weight exp(lse_k - lse) per piece; thread = head dim; every
+        // row's loads of two pieces in flight together
+        float lt[NR], acc[NR];
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+            lt[r] = (r < rb.rows_valid) ? misc->mlse[r] : -INFINITY;
+            acc[r] = 0.f;
+        }
+        for (int k0 = 0; k0 < nm; k0 += 2) {
+            float lw[2][NR], xv[2][NR];
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const bool has = k0 + jj < nm;
+                const long long sl = has ? slot_of(k0 + jj) : 0;
+#pragma unroll
+                for (int r = 0; r < NR; ++r) {
+                    const bool live = has && lt[r] != -INFINITY;
+                    lw[jj][r] = live ? __ldcg(p.part_lse + sl * RW + r) : -INFINITY;
+                    xv[jj][r] = live ? __ldcg(p.part_o + (sl * RW + r) * C::D + kl) : 0.f;
+                }
+            }
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+                for (int r = 0; r < NR; ++r)
+                    if (lw[jj][r] != -INFINITY) acc[r] += __expf(lw[jj][r] - lt[r]) * xv[jj][r];
+        }
+#pragma unroll
+        for (int r = 0; r < NR; ++r)
+            if (r < rb.rows_valid) p.out[(rb.q_row0 + r) * C::D + kl] = __float2bfloat16_rn(acc[r]);
+        if (et == 0) p.counters[sg.w] = 0;
+        // the shared merge fields are free again once every thread is past them
+        return sync();
+    };
 
     if (warp < 4) {
         // ------------------------------------------------------------ Q / K producer
@@ -399,8 +579,8 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 ptx::umma_commit(bar(C::B_SFULL + (gg & 1u)));
             };
             // O' (+)= V(gg)^T P'(gg): A = the V tile read MN-major (M = head dims), B = P'^T (K-major)
-            auto issue_pv = [&](uint32_t gg, bool first, int seg) -> bool {
-                return dec_issue_pv<C>(p, wmisc, bar0, sbase, tmem, gg, first, seg);
+            auto issue_pv = [&](uint32_t gg, bool first, int seg, bool last) -> bool {
+                return dec_issue_pv<C>(p, wmisc, bar0, sbase, tmem, gg, first, seg, last);
             };
             bool have_prev = false, prev_first = false;
             uint32_t prev_g = 0;
@@ -409,7 +589,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (sg.t1 <= sg.t0) continue;
                 // the previous segment's last PV' goes out before this segment's Q is awaited
                 if (have_prev) {
-                    ok = issue_pv(prev_g, prev_first, prev_seg);
+                    ok = issue_pv(prev_g, prev_first, prev_seg, true);
                     if (!ok) break;
                     have_prev = false;
                 }
@@ -426,7 +606,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     ptx::umma_commit(bar(C::B_KEMPTY + stk));
                     if (t == sg.t1 - 1) ptx::umma_commit(bar(C::B_QEMPTY + qb));
                     if (have_prev) {
-                        ok = issue_pv(prev_g, prev_first, prev_seg);
+                        ok = issue_pv(prev_g, prev_first, prev_seg, false);
                         if (!ok) break;
                     }
                     have_prev = true;
@@ -436,14 +616,14 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 ++seg_i;
             }
-            if (ok && have_prev) ok = issue_pv(prev_g, prev_first, prev_seg);
+            if (ok && have_prev) ok = issue_pv(prev_g, prev_first, prev_seg, true);
             ptx::umma_commit(bar(C::B_FINAL));
             drain_bar(bar(C::B_FINAL), 1, p.timeout_cycles);
         }
-        // ------------------------------------------------------------ ticket taker
+        // ------------------------------------------------------------ span bounds
         else if (warp == 3) {
             // the whole warp fills the span bounds of every CTA (the tickets and the
-            // merges look other CTAs' spans up there), then lane 0 takes the tickets
+            // merges look other CTAs' spans up there)
             if (p.B <= kMaxWeightedB) {
                 fill_span_bounds(p, misc->yb, NC, misc->bounds);
             } else {
@@ -452,26 +632,6 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 __syncwarp();
             }
             if (lane == 0) ptx::mbar_arrive(bar(C::B_BOUNDS));
-        }
-        if (warp == 3 && lane == 0) {
-            SegWalker wk;
-            wk.init(p, misc->span, cta);
-            Seg sg;
-            int j = 0;
-            while (j < 2 && wk.next(p, sg)) {
-                if (sg.kind != 1) continue;
-                if (!wait_bar(bar(C::B_MJOB + j), 0, wmisc, p)) break;
-                const int* bd = misc->bounds;
-                const int c_first = cta_of_table(bd, NC, sg.pw);
-                const int c_last = cta_of_table(bd, NC, sg.pw + sg.ntiles - 1);
-                int ncontrib = 0;
-                for (int cc = c_first; cc <= c_last; ++cc) ncontrib += bd[cc] < bd[cc + 1];
-                __threadfence();
-                const int old = atomicAdd(p.counters + sg.w, 1);
-                misc->ticket[j] = (old == ncontrib - 1);
-                ptx::mbar_arrive(bar(C::B_MTICK + j));
-                ++j;
-            }
         }
     }
     // ---------------------------------------------------------------- softmax warps
@@ -512,7 +672,6 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         Seg sg;
         uint32_t g = 0;
         bool ok = true;
-        int njob = 0;
         int seg_i = 0;
         // P'^T address of this thread's key in a P' buffer: row r adds r*128 and
         // swizzles the 16-byte chunk by r % 8
@@ -580,7 +739,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         okw = __all_sync(0xffffffffu, okw);
                         if (!okw) { ok = false; break; }
                         ptx::tc_fence_after();
-                        const uint32_t to = tmem + lane_off + C::TM_O;
+                        const uint32_t to = tmem + lane_off + C::tm_o(seg_i & 1);
                         uint32_t o[NR];
                         if constexpr (NR == 16) ptx::tmem_ld16(to, o);
                         else ptx::tmem_ld8(to, o);
@@ -632,180 +791,83 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             if (!ok) break;
 
-            // ------------------------------------------------ segment epilogue
+            // ------------------------------------------------ segment end
+            // The row statistics go to shared memory; the epilogue (the epilogue
+            // warps, or these warps with FP8 K/V) finishes the segment from O'(seg % 2).
             {
-                bool okw = wait_bar(bar(C::B_PVDONE + ((g - 1) & 1u)), ((g - 1) >> 1) & 1u, wmisc, p);
-                okw = __all_sync(0xffffffffu, okw);
-                if (!okw) { ok = false; break; }
-                ptx::tc_fence_after();
-            }
-            float lsum[NR];
-            ok = cta_reduce(l_t, lsum, false);
-            if (!ok) break;
-            uint32_t o[NR];
-            {
-                const uint32_t to = tmem + lane_off + C::TM_O;
-                if constexpr (NR == 16) ptx::tmem_ld16(to, o);
-                else ptx::tmem_ld8(to, o);
-                ptx::tmem_wait_ld();
-            }
-            // O' is read: the next segment's first PV' may overwrite it
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar(C::B_OFREE));
-            const bool direct = (sg.kind == 0);
-            // The row loop is rolled: this code first runs while every SM streams K/V,
-            // and each of its instruction-cache lines is fetched then (fewer lines,
-            // shorter stall).  It reads copies of the row state, so the arrays the tile
-            // loop uses stay in registers.
-            float em[NR], el[NR], eo[NR];
+                float lsum[NR];
+                ok = cta_reduce(l_t, lsum, false);
+                if (!ok) break;
+                const int ob = seg_i & 1;
+                // the epilogue of the segment two back has read this statistics slot
+                if (seg_i >= 2) {
+                    ok = __all_sync(0xffffffffu, wait_bar(bar(C::B_OFREE + ob), ((seg_i - 2) >> 1) & 1, wmisc, p));
+                    if (!ok) break;
+                }
+                // thread r < NR finishes row r: the factor O' is scaled by and the lse
+                // (with the sink for a direct segment; a split piece's own lse otherwise)
+                if (stid < NR) {
+                    float mr = 0.f, lr = 0.f;
 #pragma unroll
-            for (int r = 0; r < NR; ++r) {
-                em[r] = m_run[r];
-                el[r] = lsum[r];
-                eo[r] = __uint_as_float(o[r]);
-            }
-#pragma unroll 1
-            for (int r = 0; r < NR; ++r) {
-                if (r >= rb.rows_valid) break;
-                const long long fr = rb.q_row0 + r;  // flat row (b*Hq + h)*Tq + i
-                float w = 0.f, lse_v = -INFINITY;
-                if (direct) {
-                    const int h = rb.g * p.G + r / p.Tq;
-                    const float sk = (p.sink != nullptr) ? __ldg(p.sink + h) * LOG2E : -INFINITY;
-                    const float M = fmax_nan(em[r], sk);
-                    if (M != -INFINITY) {
-                        const float a = pos_or_nan(el[r]) ? ptx::ex2(em[r] - M) : 0.f;
-                        const float lt = el[r] * a + ((sk != -INFINITY) ? ptx::ex2(sk - M) : 0.f);
-                        if (pos_or_nan(lt)) {
-                            w = a / lt * p.v_scale;
-                            lse_v = (M + __log2f(lt)) * LN2;
+                    for (int r = 0; r < NR; ++r)
+                        if (stid == r) {
+                            mr = m_run[r];
+                            lr = lsum[r];
+                        }
+                    float w = 0.f, lse_v = -INFINITY;
+                    if (stid < rb.rows_valid) {
+                        if (sg.kind == 0) {
+                            const int h = rb.g * p.G + stid / p.Tq;
+                            const float sk = (p.sink != nullptr) ? __ldg(p.sink + h) * LOG2E : -INFINITY;
+                            const float M = fmax_nan(mr, sk);
+                            if (M != -INFINITY) {
+                                const float a = pos_or_nan(lr) ? ptx::ex2(mr - M) : 0.f;
+                                const float lt = lr * a + ((sk != -INFINITY) ? ptx::ex2(sk - M) : 0.f);
+                                if (pos_or_nan(lt)) {
+                                    w = a / lt * p.v_scale;
+                                    lse_v = (M + __log2f(lt)) * LN2;
+                                }
+                            }
+                        } else if (pos_or_nan(lr)) {
+                            w = p.v_scale / lr;
+                            lse_v = (mr + __log2f(lr)) * LN2;
                         }
                     }
-                    p.out[fr * C::D + kl] = __float2bfloat16_rn(w != 0.f ? eo[r] * w : 0.f);
-                    if (kl == 0 && p.lse != nullptr) p.lse[fr] = lse_v;
-                } else {
-                    if (pos_or_nan(el[r])) {
-                        w = p.v_scale / el[r];
-                        lse_v = (em[r] + __log2f(el[r])) * LN2;
-                    }
-                    const long long prow = static_cast<long long>(sg.slot) * BM + r;
-                    __stcg(p.part_o + prow * C::D + kl, w != 0.f ? eo[r] * w : 0.f);
-                    if (kl == 0) __stcg(p.part_lse + prow, lse_v);
+                    misc->seg_w[ob][stid] = w;
+                    misc->seg_lse[ob][stid] = lse_v;
                 }
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar(C::B_STATS + ob));
             }
-            // a split segment's partial rows are written
-            if (!xsync()) { ok = false; break; }
-            if (sg.kind == 1 && njob < 2) {
-                if (stid == 0) {
-                    misc->jobs[njob] = sg;
-                    ptx::mbar_arrive(bar(C::B_MJOB + njob));
-                }
-                ++njob;
+            if constexpr (!C::EPIW) {
+                ok = epi_segment(sg, seg_i, quad, xsync);
+                if (!ok) break;
             }
             ++seg_i;
         }
-        // merges of the row-blocks whose last piece this CTA wrote
-        for (int j = 0; ok && j < njob; ++j) {
-            ok = wait_bar(bar(C::B_MTICK + j), 0, wmisc, p);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            if (!misc->ticket[j]) continue;
-            ok = __all_sync(0xffffffffu, wait_bar(bar(C::B_BOUNDS), 0, wmisc, p));
-            if (!ok) break;
-            __threadfence();
-            const Seg sgm = misc->jobs[j];
-            const RB rb = rb_of(p, sgm.w);
-            const int* bd = misc->bounds;
-            const int c_first = cta_of_table(bd, NC, sgm.pw);
-            const int c_last = cta_of_table(bd, NC, sgm.pw + sgm.ntiles - 1);
-            const bool c0_first = bd[c_first] == sgm.pw;
-            const long long RW = BM;
-            if (warp == 4) {
-                int nm = 0;
-                for (int base = c_first; base <= c_last; base += 32) {
-                    const int cc = base + lane;
-                    const bool has = cc <= c_last && bd[cc] < bd[cc + 1];
-                    const unsigned m = __ballot_sync(0xffffffffu, has);
-                    const int k = nm + __popc(m & ((1u << lane) - 1u));
-                    if (has && k < kMaxMergeSlots) misc->mslot[k] = static_cast<int>(merge_slot(cc, c_first, c0_first));
-                    nm += __popc(m);
-                }
-                if (lane == 0) misc->nmerge = nm;
-            }
-            if (!xsync()) { ok = false; break; }
-            const int nm = misc->nmerge;
-            auto slot_of = [&](int k) -> long long {  // k-th contributing CTA's slot
-                if (nm <= kMaxMergeSlots) return misc->mslot[k];
-                int seen = 0;
-                for (int cc = c_first; cc <= c_last; ++cc) {
-                    if (!(bd[cc] < bd[cc + 1])) continue;
-                    if (seen++ == k) return merge_slot(cc, c_first, c0_first);
-                }
-                return 0;
-            };
-            // lse of each merged row (the sink enters here, once); eight pieces' loads at a time
-            for (int r = stid; r < rb.rows_valid; r += NSOFT_DEC) {
-                const int hr = rb.g * p.G + r / p.Tq;
-                const float sk = (p.sink != nullptr) ? __ldg(p.sink + hr) : -INFINITY;
-                float Lx = sk, z = 0.f;
-                for (int k0 = 0; k0 < nm; k0 += 8) {
-                    float lv[8];
-#pragma unroll
-                    for (int jj = 0; jj < 8; ++jj)
-                        lv[jj] = (k0 + jj < nm) ? __ldcg(p.part_lse + slot_of(k0 + jj) * RW + r) : -INFINITY;
-                    float mx = Lx;
-#pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) mx = fmax_nan(mx, lv[jj]);
-                    if (mx != -INFINITY) {
-                        // running (max, sum) over the pieces seen so far
-                        z = (Lx != -INFINITY) ? z * __expf(Lx - mx) : 0.f;
-#pragma unroll
-                        for (int jj = 0; jj < 8; ++jj) z += __expf(lv[jj] - mx);
-                        Lx = mx;
-                    }
-                }
-                float ltr = -INFINITY;
-                if (Lx != -INFINITY) {
-                    if (sk != -INFINITY) z += __expf(sk - Lx);
-                    ltr = Lx + __logf(z);
-                }
-                misc->mlse[r] = ltr;
-                if (p.lse != nullptr) p.lse[rb.q_row0 + r] = ltr;
-            }
-            if (!xsync()) { ok = false; break; }
-            // O rows: weight exp(lse_k - lse) per piece; thread = head dim; every
-            // row's loads of two pieces in flight together
-            float lt[NR], acc[NR];
-#pragma unroll
-            for (int r = 0; r < NR; ++r) {
-                lt[r] = (r < rb.rows_valid) ? misc->mlse[r] : -INFINITY;
-                acc[r] = 0.f;
-            }
-            for (int k0 = 0; k0 < nm; k0 += 2) {
-                float lw[2][NR], xv[2][NR];
-#pragma unroll
-                for (int jj = 0; jj < 2; ++jj) {
-                    const bool has = k0 + jj < nm;
-                    const long long sl = has ? slot_of(k0 + jj) : 0;
-#pragma unroll
-                    for (int r = 0; r < NR; ++r) {
-                        const bool live = has && lt[r] != -INFINITY;
-                        lw[jj][r] = live ? __ldcg(p.part_lse + sl * RW + r) : -INFINITY;
-                        xv[jj][r] = live ? __ldcg(p.part_o + (sl * RW + r) * C::D + kl) : 0.f;
-                    }
-                }
-#pragma unroll
-                for (int jj = 0; jj < 2; ++jj)
-#pragma unroll
-                    for (int r = 0; r < NR; ++r)
-                        if (lw[jj][r] != -INFINITY) acc[r] += __expf(lw[jj][r] - lt[r]) * xv[jj][r];
-            }
-#pragma unroll
-            for (int r = 0; r < NR; ++r)
-                if (r < rb.rows_valid) p.out[(rb.q_row0 + r) * C::D + kl] = __float2bfloat16_rn(acc[r]);
-            if (stid == 0) p.counters[sgm.w] = 0;
-            if (!xsync()) { ok = false; break; }
+    }
+    // ---------------------------------------------------------------- epilogue warps
+    else if constexpr (C::EPIW) {
+        const int quad = warp & 3;
+        uint32_t eph = 0;
+        auto esync = [&]() -> bool {  // the four epilogue warps, bounded
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(C::B_ESYNC));
+            const bool r = wait_bar(bar(C::B_ESYNC), eph & 1, wmisc, p);
+            ++eph;
+            ptx::tc_fence_after();
+            return __all_sync(0xffffffffu, r);
+        };
+        SegWalker wk;
+        wk.init(p, misc->span, cta);
+        Seg sg;
+        int seg_i = 0;
+        bool ok = true;
+        while (ok && wk.next(p, sg)) {
+            if (sg.t1 <= sg.t0) continue;
+            ok = epi_segment(sg, seg_i, quad, esync);
+            ++seg_i;
         }
     }
 

@@ -379,7 +379,10 @@ def _wide(segs, nbox, vch, nslot, rnd, mutate=False):
 # swap-AB decode kernel (head dim 128, at most 16 packed rows): gqa_dec_kernel
 
 
-def _decode(segs, stk, stv, rnd):
+def _decode(segs, stk, stv, rnd, epiw=True, mutate=False):
+    """epiw: the segment epilogues run on their own warpgroup (bf16 K/V);
+    otherwise the softmax warps run each one right after the segment (FP8 K/V,
+    whose warps 8-11 convert tiles)."""
     bars = {}
 
     def mk(name, count):
@@ -391,22 +394,23 @@ def _decode(segs, stk, stv, rnd):
         mk("SF%d" % i, 1)
         mk("PF%d" % i, 4)
         mk("PD%d" % i, 1)
-        mk("MJ%d" % i, 1)
-        mk("MT%d" % i, 1)
+        mk("OF%d" % i, 4)   # epilogue has read O' buffer i and its row statistics
+        mk("ST%d" % i, 4)   # softmax has written the row statistics of buffer i
+        mk("SP%d" % i, 1)   # a segment's last PV' into buffer i completed
     for i in range(stk):
         mk("KF%d" % i, 1)
         mk("KE%d" % i, 1)
     for i in range(stv):
         mk("VF%d" % i, 1)
         mk("VE%d" % i, 1)
-    mk("OFREE", 4)
     mk("RED", 4)
     mk("X", 4)
+    mk("E", 4)
+    mk("BOUNDS", 1)
     # decisions every softmax warp takes alike (they follow the CTA-wide row maxima)
     grow = [[rnd.random() < 0.3 for _ in range(n)] for n, _ in segs]
     tail = [[rnd.random() < 0.3 for _ in range(n)] for n, _ in segs]
     merges = [rnd.random() < 0.5 for _ in segs]
-    nsplit = min(2, sum(1 for _, k in segs if k == 1))
 
     def kprod():
         g = 0
@@ -426,32 +430,51 @@ def _decode(segs, stk, stv, rnd):
                 yield ("tma", ["VF%d" % (g % stv)])
                 g += 1
 
+    def bounds():
+        yield ("arrive", "BOUNDS")
+
     def mma():
-        def pv(gg, first, seg):
+        def pv(gg, first, seg, last):
             yield ("wait", "PF%d" % (gg % 2), gg // 2)
             yield ("wait", "VF%d" % (gg % stv), gg // stv)
-            if first and seg > 0:
-                yield ("wait", "OFREE", seg - 1)
-            yield ("mma", ["PD%d" % (gg % 2), "VE%d" % (gg % stv)])
+            if first and seg >= 2:
+                yield ("wait", "OF%d" % (seg % 2), (seg - 2) // 2)
+            yield ("mma", ["PD%d" % (gg % 2), "VE%d" % (gg % stv)] + (["SP%d" % (seg % 2)] if last else []))
 
         g = 0
         prev = None
         for si, (n, _) in enumerate(segs):
             if prev is not None:
-                yield from pv(*prev)
+                yield from pv(*prev, True)
                 prev = None
             yield ("wait", "QF%d" % (si % 2), si // 2)
             for t in range(n):
                 yield ("wait", "KF%d" % (g % stk), g // stk)
                 yield ("mma", ["SF%d" % (g % 2), "KE%d" % (g % stk)] + (["QE%d" % (si % 2)] if t == n - 1 else []))
                 if prev is not None:
-                    yield from pv(*prev)
+                    yield from pv(*prev, False)
                 prev = (g, t == 0, si)
                 g += 1
         if prev is not None:
-            yield from pv(*prev)
+            yield from pv(*prev, True)
 
     ph = {}
+    # the statistics slots: the segment each epilogue warp last read from slot b
+    read = [[-2] * 4 for _ in range(2)]
+
+    def epilogue(w, si, kind, sync):
+        yield ("wait", "ST%d" % (si % 2), si // 2)
+        yield ("wait", "SP%d" % (si % 2), si // 2)
+        read[si % 2][w] = si  # O' buffer and statistics read, then released
+        yield ("arrive", "OF%d" % (si % 2))
+        if kind == 1:
+            yield from sync()
+            if w == 0:
+                yield ("wait", "BOUNDS", 0)
+            yield from sync()
+            if merges[si]:
+                for _ in range(3):
+                    yield from sync()
 
     def softmax(w):
         ph[w] = {"RED": 0, "X": 0}
@@ -462,7 +485,6 @@ def _decode(segs, stk, stv, rnd):
             ph[w][name] += 1
 
         g = 0
-        njob = 0
         for si, (n, kind) in enumerate(segs):
             for t in range(n):
                 yield ("wait", "SF%d" % (g % 2), g // 2)
@@ -475,28 +497,32 @@ def _decode(segs, stk, stv, rnd):
                     yield ("wait", "VF%d" % (g % stv), g // stv)
                 yield ("arrive", "PF%d" % (g % 2))
                 g += 1
-            yield ("wait", "PD%d" % ((g - 1) % 2), (g - 1) // 2)
             yield from sync("RED")
-            yield ("arrive", "OFREE")
-            yield from sync("X")
-            if kind == 1 and njob < 2:
-                if w == 0:
-                    yield ("arrive", "MJ%d" % njob)
-                njob += 1
-        for j in range(njob):
-            yield ("wait", "MT%d" % j, 0)
-            if merges[j]:
-                for _ in range(3):
-                    yield from sync("X")
+            if si >= 2 and not mutate:
+                yield ("wait", "OF%d" % (si % 2), (si - 2) // 2)
+            # writing slot si % 2 while an epilogue warp has not read segment si - 2 from it
+            if si >= 2 and min(read[si % 2]) < si - 2:
+                raise ProtocolError("statistics slot %d overwritten before segment %d was read" % (si % 2, si - 2))
+            yield ("arrive", "ST%d" % (si % 2))
+            if not epiw:
+                yield from epilogue(w, si, kind, lambda: sync("X"))
 
-    def tickets():
-        for j in range(nsplit):
-            yield ("wait", "MJ%d" % j, 0)
-            yield ("arrive", "MT%d" % j)
+    def epi_warp(w):
+        ph[("e", w)] = 0
 
-    roles = {"kprod": kprod(), "vprod": vprod(), "mma": mma(), "tickets": tickets()}
+        def sync():
+            yield ("arrive", "E")
+            yield ("wait", "E", ph[("e", w)])
+            ph[("e", w)] += 1
+
+        for si, (n, kind) in enumerate(segs):
+            yield from epilogue(w, si, kind, sync)
+
+    roles = {"kprod": kprod(), "vprod": vprod(), "mma": mma(), "bounds": bounds()}
     for w in range(4):
         roles["softmax%d" % w] = softmax(w)
+        if epiw:
+            roles["epilogue%d" % w] = epi_warp(w)
     _simulate(bars, roles, rnd)
 
 
@@ -533,9 +559,25 @@ def test_model_catches_the_wide_tail_wait_without_the_release_wait():
     assert caught > 0
 
 
-def test_decode_protocol_has_no_deadlock_or_aliasing():
+@pytest.mark.parametrize("epiw", [True, False])
+def test_decode_protocol_has_no_deadlock_or_aliasing(epiw):
     for trial, segs, stk, stv in _layouts(5, 400):
-        _decode(segs, stk, stv, random.Random(trial))
+        _decode(segs, stk, stv, random.Random(trial), epiw=epiw)
+
+
+def test_model_catches_the_decode_statistics_written_before_their_slot_is_free():
+    """Without the softmax's wait for the epilogue two segments back, the
+    statistics barrier can run two phases ahead of the epilogue warps."""
+    caught = 0
+    rnd = random.Random(29)
+    for trial in range(1000):
+        # short split segments: the softmax runs ahead of the epilogue warps
+        segs = [(rnd.randint(1, 2), 1) for _ in range(6)]
+        try:
+            _decode(segs, 3, 3, random.Random(trial), epiw=True, mutate=True)
+        except ProtocolError:
+            caught += 1
+    assert caught > 0
 
 
 def test_model_catches_a_wrong_wait_index():
