@@ -312,13 +312,15 @@ __device__ int weighted_bound(const Params& p, const int* yb, int NC, int k, int
 }
 
 // One full warp: the batch table yb[0..B] and this CTA's SpanStart.
-__device__ void plan_span_weighted(const Params& p, int c, int NC, SpanStart* out, int* yb) {
+__device__ void plan_span_weighted(const Params& p, int c, int NC, SpanStart* out, int* yb, int* lens = nullptr) {
     const int lane = threadIdx.x & 31;
     const int E = p.seg_w;
     int acc = 0;
     for (int base = 0; base < p.B; base += 32) {
         const int bb = base + lane;
-        const int lw = bb < p.B ? p.Hkv * (qtile_ntiles(p, 0, load_len(p, bb)) + E) : 0;
+        const int n = bb < p.B ? load_len(p, bb) : 0;
+        if (lens != nullptr && bb < p.B) lens[bb] = n;
+        const int lw = bb < p.B ? p.Hkv * (qtile_ntiles(p, 0, n) + E) : 0;
         int inc = lw;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -371,8 +373,10 @@ struct SegWalker {
     long long remaining, pos;
     bool first, single_done;
     int c;
+    const int* lens;  // the batches' logical lengths in shared memory, or null (read them from global)
 
-    __device__ void init(const Params& p, const SpanStart& s, int cta) {
+    __device__ void init(const Params& p, const SpanStart& s, int cta, const int* len_table = nullptr) {
+        lens = len_table;
         w = s.w;
         t = s.t;
         remaining = (p.mode == 0) ? s.p1 - s.p0 : 0;
@@ -399,7 +403,7 @@ struct SegWalker {
         }
         if (remaining <= 0) return false;
         const int u = w / p.QW, qt = w % p.QW;
-        const int n = load_len(p, u / p.Hkv);
+        const int n = lens ? lens[u / p.Hkv] : load_len(p, u / p.Hkv);
         const int nt = qtile_ntiles(p, qt, n);
         long long take = nt - t;
         if (take > remaining) take = remaining;

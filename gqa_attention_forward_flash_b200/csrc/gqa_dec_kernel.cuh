@@ -96,7 +96,7 @@ struct DecCfg {
     // the control block holds float4-read arrays: 128-byte aligned whatever NBAR is
     static constexpr int OFF_MISC = (OFF_BAR + NBAR * 8 + 127) & ~127;
     static_assert(OFF_MISC % 128 == 0, "control block alignment");
-    static constexpr int MISC_BYTES = 1536 + 4 * (kMaxGrid + 1) + 4 * (kMaxWeightedB + 1);
+    static constexpr int MISC_BYTES = 1536 + 4 * (kMaxGrid + 1) + 4 * (kMaxWeightedB + 1) + 4 * kMaxWeightedB;
     static constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static constexpr uint32_t TM_COLS = 64;
@@ -167,6 +167,7 @@ struct DecMisc {
     int etk;                  // the epilogue's split piece completed its row-block (it merges)
     int bounds[kMaxGrid + 1];  // flat start of every CTA's span (cost-weighted), bounds[NC] = tot
     int yb[kMaxWeightedB + 1]; // weighted start of every batch (the plan's table)
+    int lens[kMaxWeightedB];   // every batch's logical length (the plan's reads, kept for the walkers)
 };
 
 // Reduce NR per-thread values over the 32 lanes of a warp, one row per lane group:
@@ -299,7 +300,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ptx::tmem_relinquish();
     }
     if (warp == 0) {
-        if (p.B <= kMaxWeightedB) plan_span_weighted(p, cta, NC, &misc->span, misc->yb);
+        if (p.B <= kMaxWeightedB) plan_span_weighted(p, cta, NC, &misc->span, misc->yb, misc->lens);
         else plan_span(p, cta, NC, &misc->span);  // equal spans (the host sets seg_w = 0)
     }
     if (warp >= 4 && warp < 8) {
@@ -488,7 +489,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint64_t pol_q = ptx::policy_evict_last();
             const uint64_t pol_kv = ptx::policy_evict_first();
             SegWalker wk;
-            wk.init(p, misc->span, cta);
+            wk.init(p, misc->span, cta, p.B <= kMaxWeightedB ? misc->lens : nullptr);
             Seg sg;
             int seg_i = 0;
             uint32_t g = 0;
@@ -531,7 +532,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         else if (warp == 1 && lane == 0) {
             const uint64_t pol_kv = ptx::policy_evict_first();
             SegWalker wk;
-            wk.init(p, misc->span, cta);
+            wk.init(p, misc->span, cta, p.B <= kMaxWeightedB ? misc->lens : nullptr);
             Seg sg;
             uint32_t g = 0;
             bool ok = true;
@@ -561,7 +562,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // ------------------------------------------------------------ MMA issuer
         else if (warp == 2 && lane == 0) {
             SegWalker wk;
-            wk.init(p, misc->span, cta);
+            wk.init(p, misc->span, cta, p.B <= kMaxWeightedB ? misc->lens : nullptr);
             Seg sg;
             int seg_i = 0;
             uint32_t g = 0;
@@ -668,7 +669,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             return okr;
         };
         SegWalker wk;
-        wk.init(p, misc->span, cta);
+        wk.init(p, misc->span, cta, p.B <= kMaxWeightedB ? misc->lens : nullptr);
         Seg sg;
         uint32_t g = 0;
         bool ok = true;
@@ -860,7 +861,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             return __all_sync(0xffffffffu, r);
         };
         SegWalker wk;
-        wk.init(p, misc->span, cta);
+        wk.init(p, misc->span, cta, p.B <= kMaxWeightedB ? misc->lens : nullptr);
         Seg sg;
         int seg_i = 0;
         bool ok = true;
@@ -875,7 +876,7 @@ gqa_dec_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     else if constexpr (C::FP8) {
         const int ct = threadIdx.x - 256;  // 0..127
         SegWalker wk;
-        wk.init(p, misc->span, cta);
+        wk.init(p, misc->span, cta, p.B <= kMaxWeightedB ? misc->lens : nullptr);
         Seg sg;
         int seg_i = 0;
         uint32_t g = 0;
