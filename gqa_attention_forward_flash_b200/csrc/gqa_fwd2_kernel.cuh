@@ -266,8 +266,12 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ptx::regs_dec<88>();
         // ------------------------------------------------------------ producers
         if (warp == 8 && lane == 0) {
-            const uint64_t pol_q = ptx::policy_evict_last();
-            const uint64_t pol_kv = (p.QW == 1) ? ptx::policy_evict_first() : ptx::policy_evict_normal();
+            // one row-block per KV head (QW == 1): Q serves every tile and K/V stream
+            // once; several row-blocks per KV head (prefill): each Q tile is read once
+            // and every row-block of the head reads the head's K/V again, so K/V stay
+            // in L2 ahead of Q (and of O, written with a streaming hint)
+            const uint64_t pol_q = (p.QW == 1) ? ptx::policy_evict_last() : ptx::policy_evict_first();
+            const uint64_t pol_kv = (p.QW == 1) ? ptx::policy_evict_first() : ptx::policy_evict_last();
             SegWalker wk;
             wk.init(p, misc->span, cta);
             Seg sg;
@@ -304,7 +308,7 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int i = 0; i < C::STK; ++i) drain_bar(bar(C::B_KFULL + i), k_issued[i], p.timeout_cycles);
             drain_bar(bar(C::B_QFULL), q_issued, p.timeout_cycles);
         } else if (warp == 11 && lane == 0) {
-            const uint64_t pol_kv = (p.QW == 1) ? ptx::policy_evict_first() : ptx::policy_evict_normal();
+            const uint64_t pol_kv = (p.QW == 1) ? ptx::policy_evict_first() : ptx::policy_evict_last();
             SegWalker wk;
             wk.init(p, misc->span, cta);
             Seg sg;
@@ -743,9 +747,9 @@ gqa_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             uint4* d4 = reinterpret_cast<uint4*>(p.out + fr * C::D + c0 + c * 32);
 #pragma unroll
                             for (int j = 0; j < 4; ++j)
-                                d4[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
-                                                   pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
-                                                   pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+                                __stcs(d4 + j, make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                                                          pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
+                                                          pack_bf16x2(v[8 * j + 6], v[8 * j + 7])));
                         } else {
                             float4* d4 = reinterpret_cast<float4*>(pdst + c * 32);
 #pragma unroll
