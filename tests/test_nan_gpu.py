@@ -17,6 +17,7 @@ that see the key, the rows of the same 128-key tile that mask it by causality
 """
 import numpy as np
 import pytest
+import torch
 
 from gqa_attention_forward_flash_b200.synth import Workload, make_inputs
 
@@ -58,3 +59,30 @@ def test_nan_in_visible_key_or_value_poisons_exactly_the_rows_that_see_it(name):
     assert np.array_equal(np.isnan(l), np.isnan(l_ref)), "%s: NaN lse rows differ" % name
     keep = ~nan_ref
     compare(o[keep], l[keep], o_ref[keep], l_ref[keep], name)
+
+
+@pytest.mark.parametrize("which", ["k8", "v8"])
+def test_nan_in_visible_fp8_byte_poisons_exactly_the_rows_that_see_it(which):
+    """E4M3 K/V (the decode kernel's FP8 variant, whose softmax warps run the
+    segment epilogues themselves): the NaN code 0x7F inside a row's visible
+    keys makes exactly the rows that see it NaN, as in the oracle's decode."""
+    import oracle
+    from gqa_attention_forward_flash_b200 import binding
+
+    w = Workload("nan_fp8", B=3, Hq=32, Hkv=4, Tq=1, Tkv=1500, d=128, kv_fp8=True, seed=37)
+    inp = make_inputs(w)
+    getattr(inp, which).view(torch.uint8)[1, 2, 700, 5] = 0x7F  # the E4M3 NaN code
+    dev = "cuda"
+    out, lse = binding.gqa_attention_fwd_fp8kv(inp.q.to(dev), inp.k8.to(dev), inp.v8.to(dev), inp.k_scale,
+                                               inp.v_scale, None, None, scale=inp.scale, causal=inp.causal)
+    assert binding.gqa_get_device_error() == 0
+    o = out.float().cpu().numpy().astype(np.float64)
+    l = lse.cpu().numpy().astype(np.float64)
+    ro, rl = oracle.attention_fp8kv(inp.q, inp.k8, inp.v8, inp.k_scale, inp.v_scale, None, None,
+                                    scale=inp.scale, causal=inp.causal)
+    nan_ref = np.isnan(ro).any(axis=-1)
+    assert nan_ref.any() and not nan_ref.all()
+    assert np.array_equal(np.isnan(o).any(axis=-1), nan_ref)
+    assert np.array_equal(np.isnan(l), np.isnan(rl))
+    keep = ~nan_ref
+    compare(o[keep], l[keep], ro[keep], rl[keep], "fp8 " + which)
